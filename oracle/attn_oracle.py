@@ -1,0 +1,310 @@
+"""Float64 CPU oracle for exact scaled-dot-product attention with online softmax.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` import this module. The product path (the
+CUDA library and its Python binding) never calls it, and it calls nothing of
+the product path: it shares no code, table or constant with the kernels.
+
+What it computes, and the passages it follows:
+
+* Exact attention O = softmax(Q K^T * scale + mask) V, materialised. The
+  method is exact, not an approximation ("flash-attention与TensorRT-LLM集成",
+  section 背景与痛点分析, which names the paper "FlashAttention: Fast and
+  Memory-Efficient Exact Attention with IO-Awareness"; "LLM推理优化技术综述",
+  PART04). The log-sum-exp LSE = max + ln(sum exp(s - max)) is returned beside
+  O in natural-log units.
+* Grouped-query head mapping: query head h reads KV head floor(h / G) with
+  G = Hq / Hkv, the mapping that duplicating each KV head G times produces
+  ("TensorRT对Grouped Query Attention的支持进展", sections 技术演进背景 and
+  图优化与算子融合; "LLM推理优化技术综述", PART03). MHA is G = 1, MQA is Hkv = 1.
+* Causal mask: key j is visible to query i iff j <= i (autoregressive
+  generation, "LLM推理优化技术综述", PART01). Queries and keys share positions.
+* Paged KV cache: token p of a sequence lives in physical page
+  block_table[p // page_size], slot p % page_size ("LLM推理优化技术综述",
+  PART02: a block table maps contiguous logical blocks to non-contiguous
+  physical ones; "Optimizing Inference on LLMs with TensorRT-LLM", PagedAttention
+  section). The oracle gathers the pages and applies the dense formula.
+* BLASST tile skip ("高效部署稀疏注意力加速方案：BLASST方法详解与实践指南",
+  section 架构与组件: keep a running maximum of the attention scores during the
+  blockwise online softmax and compare against a threshold lambda; a negligible
+  block skips its exponentials, its Value load and its matrix product). The
+  pages do not print the inequality. The reading used here: a KV tile of 64
+  keys is skipped iff lambda > 0 and, for every row of the decision unit,
+  exp(tile_rowmax - running_max) < lambda (strict), on scaled natural-log
+  scores, where running_max is the maximum over the tiles of the unit already
+  kept. A row that sees no key of the tile is vacuously below the threshold;
+  a row whose running maximum is still -inf is not. The walk visits the tiles
+  of a unit in ascending key order; the result is the exact formula
+  restricted to the kept keys.
+
+Parity status: dense prefill, paged decode and the gather are pinned by the
+CPU tests (brute force, torch's float64 SDPA, closed forms, invariants). The
+BLASST walk is pinned against a brute-force recomputation of the rule from the
+full score matrix and against its invariants; the rule itself is a reading of
+the pages ("parity unpinned" against the pages, which never print it).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+NEG_INF = -np.inf
+KV_TILE = 64          # keys per BLASST decision tile (block_size 64 in the BLASST guide's config)
+Q_TILE = 128          # query rows per prefill decision unit
+
+
+def _f64(x):
+    """Widen a tensor or array (bf16 torch tensors included) to float64 numpy."""
+    if hasattr(x, "detach"):
+        return x.detach().to("cpu").double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def kv_head_of(hq: int, Hq: int, Hkv: int) -> int:
+    """Query head hq reads KV head floor(hq / (Hq / Hkv))."""
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return hq // (Hq // Hkv)
+
+
+def attention_rows(q, k, v, scale, visible=None):
+    """Exact attention for one head.
+
+    q [R, D], k [N, D], v [N, D] (float64); visible: bool [R, N] or None (all
+    keys visible). Returns (o [R, D], lse [R]). A row that sees no key gets
+    o = 0 and lse = -inf.
+    """
+    s = (q @ k.T) * scale
+    if visible is not None:
+        s = np.where(visible, s, NEG_INF)
+    m = s.max(axis=1) if s.shape[1] else np.full(s.shape[0], NEG_INF)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    p = np.exp(s - m_safe[:, None])                    # exp(-inf) = 0 for hidden keys
+    l = p.sum(axis=1)
+    l_safe = np.where(empty, 1.0, l)
+    o = (p @ v) / l_safe[:, None]
+    o[empty] = 0.0
+    lse = np.where(empty, NEG_INF, m_safe + np.log(l_safe))
+    return o, lse
+
+
+def causal_visible(rows, n_keys):
+    """bool [len(rows), n_keys]: key j visible to query row i iff j <= i."""
+    rows = np.asarray(rows)
+    return np.arange(n_keys)[None, :] <= rows[:, None]
+
+
+def prefill(q, k, v, causal: bool, scale: float, row_block: int = 2048,
+            heads=None, rows=None):
+    """Dense prefill attention.
+
+    q [B, S, Hq, D], k/v [B, S, Hkv, D] (any dtype; widened to float64).
+    Returns o [B, S, Hq, D] and lse [B, Hq, S] (float64). ``heads`` (list of
+    (b, hq)) and ``rows`` (list of query positions) restrict the work to a
+    sample; entries outside the sample are NaN. Row blocking only bounds
+    memory: every row still sees its full key range.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, S, Hq, _ = q.shape
+    Hkv = k.shape[2]
+    o = np.full((B, S, Hq, v.shape[-1]), np.nan)   # value width may differ from the key width
+    lse = np.full((B, Hq, S), np.nan)
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(Hq)]
+    row_list = np.arange(S) if rows is None else np.asarray(sorted(set(int(r) for r in rows)))
+    for b, hq in heads:
+        kv = kv_head_of(hq, Hq, Hkv)
+        for i0 in range(0, len(row_list), row_block):
+            rr = row_list[i0:i0 + row_block]
+            vis = causal_visible(rr, S) if causal else None
+            ob, lb = attention_rows(q[b, rr, hq, :], k[b, :, kv, :], v[b, :, kv, :], scale, vis)
+            o[b, rr, hq, :] = ob
+            lse[b, hq, rr] = lb
+    return o, lse
+
+
+def gather_pages(pages, block_table_row, seq_len: int, page_size: int):
+    """Contiguous [seq_len, Hkv, D] view of one sequence's paged K or V.
+
+    pages [P, page_size, Hkv, D]; token p is pages[block_table_row[p // page_size], p % page_size].
+    """
+    pages = _f64(pages)
+    out = np.empty((seq_len,) + pages.shape[2:])
+    for p in range(seq_len):
+        page = int(block_table_row[p // page_size])
+        if page < 0 or page >= pages.shape[0]:
+            raise IndexError(f"block_table entry {page} out of range for token {p}")
+        out[p] = pages[page, p % page_size]
+    return out
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, page_size: int, scale: float,
+                 seqs=None):
+    """Single-token decode over a paged KV cache (dense, no skip).
+
+    q [N, Hq, D]; k_pages/v_pages [P, page_size, Hkv, D]; block_table [N, max_pages]
+    int; seq_lens [N] int. The new query sees all seq_len cached keys.
+    Returns o [N, Hq, D] and lse [N, Hq] (float64); a sequence of length 0
+    gives o = 0 and lse = -inf.
+    """
+    q = _f64(q)
+    bt = np.asarray(block_table)
+    lens = np.asarray(seq_lens)
+    N, Hq, D = q.shape
+    Hkv = k_pages.shape[2]
+    o = np.full((N, Hq, D), np.nan)
+    lse = np.full((N, Hq), np.nan)
+    for b in (range(N) if seqs is None else seqs):
+        L = int(lens[b])
+        kb = gather_pages(k_pages, bt[b], L, page_size)
+        vb = gather_pages(v_pages, bt[b], L, page_size)
+        for hq in range(Hq):
+            kv = kv_head_of(hq, Hq, Hkv)
+            ob, lb = attention_rows(q[b, hq][None, :], kb[:, kv, :], vb[:, kv, :], scale)
+            o[b, hq], lse[b, hq] = ob[0], lb[0]
+    return o, lse
+
+
+# ----------------------------------------------------------------------------
+# BLASST walk
+# ----------------------------------------------------------------------------
+
+def blasst_walk(s, visible, tiles, lam: float):
+    """Run the skip decisions of one decision unit.
+
+    s [R, N] scaled scores of the unit's rows against the keys it may visit;
+    visible bool [R, N]; tiles: list of key-index ranges (start, stop) in
+    visiting order. Returns (kept bool [R, N], skipped list[bool] per tile,
+    margin list[float] per tile). ``margin`` is the smallest
+    |exp(r - m) - lam| over the rows where both r and m are finite (inf when
+    no row has both), the distance of the decision from a tie.
+    """
+    R = s.shape[0]
+    m = np.full(R, NEG_INF)
+    kept = np.zeros_like(visible)
+    skipped, margins = [], []
+    for (c0, c1) in tiles:
+        vis_t = visible[:, c0:c1]
+        any_vis = vis_t.any(axis=1)
+        r = np.where(any_vis, np.where(vis_t, s[:, c0:c1], NEG_INF).max(axis=1, initial=NEG_INF), NEG_INF)
+        both = np.isfinite(r) & np.isfinite(m)
+        ratio = np.exp(np.where(both, r - np.where(both, m, 0.0), 0.0))
+        row_ok = np.where(~np.isfinite(r), True,
+                          np.where(~np.isfinite(m), False, ratio < lam))
+        skip = bool(lam > 0.0 and row_ok.all())
+        margins.append(float(np.abs(ratio[both] - lam).min()) if both.any() else math.inf)
+        skipped.append(skip)
+        if not skip:
+            m = np.maximum(m, r)
+            kept[:, c0:c1] = vis_t
+    return kept, skipped, margins
+
+
+def _attention_kept(s, kept, v):
+    """Exact formula restricted to the kept keys (scores already scaled)."""
+    s = np.where(kept, s, NEG_INF)
+    m = s.max(axis=1)
+    p = np.exp(s - m[:, None])
+    l = p.sum(axis=1)
+    return (p @ v) / l[:, None], m + np.log(l)
+
+
+def prefill_blasst(q, k, v, causal: bool, scale: float, lam: float, heads=None, q_tiles=None):
+    """Prefill with the BLASST tile skip.
+
+    Decision unit: (b, hq, q tile of 128 rows [128 qt, min(128 qt + 128, S))).
+    Its tiles are the 64-key tiles t = 0, 1, ... in ascending order; causal
+    units visit only tiles with 64 t <= last row of the q tile.
+    Returns o [B,S,Hq,D], lse [B,Hq,S], skip [B,Hq,n_qt,n_kt] uint8
+    (1 skipped, 0 kept, 2 not visited) and margin [B,Hq,n_qt,n_kt] float64
+    (inf where not visited). ``heads``/``q_tiles`` restrict the work to a sample.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    n_qt = -(-S // Q_TILE)
+    n_kt = -(-S // KV_TILE)
+    o = np.full((B, S, Hq, D), np.nan)
+    lse = np.full((B, Hq, S), np.nan)
+    skip = np.full((B, Hq, n_qt, n_kt), 2, dtype=np.uint8)
+    margin = np.full((B, Hq, n_qt, n_kt), np.inf)
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(Hq)]
+    for b, hq in heads:
+        kv = kv_head_of(hq, Hq, Hkv)
+        for qt in (range(n_qt) if q_tiles is None else q_tiles):
+            rows = np.arange(qt * Q_TILE, min(qt * Q_TILE + Q_TILE, S))
+            last = rows[-1]
+            n_vis_tiles = (last // KV_TILE + 1) if causal else n_kt
+            n_keys = min(n_vis_tiles * KV_TILE, S)
+            s = (q[b, rows, hq, :] @ k[b, :n_keys, kv, :].T) * scale
+            vis = causal_visible(rows, n_keys) if causal else np.ones((len(rows), n_keys), bool)
+            tiles = [(t * KV_TILE, min(t * KV_TILE + KV_TILE, n_keys)) for t in range(n_vis_tiles)]
+            kept, skipped, margins = blasst_walk(s, vis, tiles, lam)
+            ob, lb = _attention_kept(s, kept, v[b, :n_keys, kv, :])
+            o[b, rows, hq, :] = ob
+            lse[b, hq, rows] = lb
+            skip[b, hq, qt, :n_vis_tiles] = np.asarray(skipped, dtype=np.uint8)
+            margin[b, hq, qt, :n_vis_tiles] = margins
+    return o, lse, skip, margin
+
+
+def decode_paged_blasst(q, k_pages, v_pages, block_table, seq_lens, page_size: int,
+                        scale: float, lam: float, split_tokens: int,
+                        rows_per_unit: str = "group", seqs=None):
+    """Paged decode with the BLASST tile skip.
+
+    Decision unit: (sequence, KV head, split). A split covers tokens
+    [sp * split_tokens, min((sp + 1) * split_tokens, L)); its tiles are its
+    64-token tiles in ascending order and its running maximum starts at -inf.
+    The unit's rows are the G query heads that share the KV head
+    (rows_per_unit="group") or each query head alone (rows_per_unit="head").
+    Returns o [N,Hq,D], lse [N,Hq], skip and margin indexed
+    [N, Hkv, max_tiles] with max_tiles = ceil(max_pages * page_size / 64)
+    (for "head": [N, Hq, max_tiles]); skip is 1 skipped, 0 kept, 2 not visited.
+    """
+    if split_tokens % KV_TILE != 0 or split_tokens <= 0:
+        raise ValueError("split_tokens must be a positive multiple of 64")
+    q = _f64(q)
+    bt = np.asarray(block_table)
+    lens = np.asarray(seq_lens)
+    N, Hq, D = q.shape
+    Hkv = k_pages.shape[2]
+    G = Hq // Hkv
+    max_tiles = -(-bt.shape[1] * page_size // KV_TILE)
+    n_units = Hkv if rows_per_unit == "group" else Hq
+    o = np.full((N, Hq, D), np.nan)
+    lse = np.full((N, Hq), np.nan)
+    skip = np.full((N, n_units, max_tiles), 2, dtype=np.uint8)
+    margin = np.full((N, n_units, max_tiles), np.inf)
+    for b in (range(N) if seqs is None else seqs):
+        L = int(lens[b])
+        if L == 0:
+            o[b], lse[b] = 0.0, NEG_INF
+            continue
+        kb = gather_pages(k_pages, bt[b], L, page_size)
+        vb = gather_pages(v_pages, bt[b], L, page_size)
+        for kv in range(Hkv):
+            heads = list(range(kv * G, kv * G + G))
+            groups = [heads] if rows_per_unit == "group" else [[h] for h in heads]
+            for rows in groups:
+                s = (q[b, rows, :] @ kb[:, kv, :].T) * scale           # [R, L]
+                kept = np.zeros(s.shape, dtype=bool)
+                unit = kv if rows_per_unit == "group" else rows[0]
+                for sp0 in range(0, L, split_tokens):
+                    sp1 = min(sp0 + split_tokens, L)
+                    tiles = [(t, min(t + KV_TILE, sp1)) for t in range(sp0, sp1, KV_TILE)]
+                    vis = np.zeros(s.shape, dtype=bool)
+                    vis[:, sp0:sp1] = True
+                    kept_sp, skipped, margins = blasst_walk(s, vis, tiles, lam)
+                    kept |= kept_sp
+                    t0 = sp0 // KV_TILE
+                    skip[b, unit, t0:t0 + len(skipped)] = np.asarray(skipped, dtype=np.uint8)
+                    margin[b, unit, t0:t0 + len(margins)] = margins
+                ob, lb = _attention_kept(s, kept, vb[:, kv, :])
+                o[b, rows, :] = ob
+                lse[b, rows] = lb
+    return o, lse, skip, margin
