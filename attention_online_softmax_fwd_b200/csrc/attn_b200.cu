@@ -1,0 +1,301 @@
+// C ABI of the attention library: argument validation, TMA descriptor
+// encoding and kernel launches. Everything is enqueued on the caller's stream;
+// nothing here allocates device memory or synchronises (except
+// attn_read_device_status, which is documented to).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+using namespace attn;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int sms = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+// Current device's SM count; ATTN_ERR_UNSUPPORTED unless it is compute capability 10.0.
+int current_device(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, count = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.sms = count;
+    d.ready = true;
+  }
+  if (!d.supported) return ATTN_ERR_UNSUPPORTED;
+  *sms = d.sms;
+  return ATTN_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor map. dims/box innermost first; strides in bytes for dims 1..3.
+int encode_map(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+               const uint32_t box[4], CUtensorMapSwizzle swizzle) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return ATTN_ERR_CUDA;
+  const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+  cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t s[3] = {strides[0], strides[1], strides[2]};
+  cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d, s, b, elem_strides,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [B][S][H][D] bf16 tensor as a 4-D map {D, S, H, B}; box = 64 columns x 128 rows of one head.
+int encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+  const uint64_t dims[4] = {uint64_t(D), uint64_t(S), uint64_t(H), uint64_t(B)};
+  const uint64_t strides[3] = {uint64_t(H) * D * 2, uint64_t(D) * 2, uint64_t(S) * H * D * 2};
+  const uint32_t box[4] = {64, uint32_t(kPfRows), 1, 1};
+  return encode_map(map, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
+
+template <int D, bool CAUSAL, bool SKIP>
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
+                   int sms, cudaStream_t stream) {
+  auto kernel = prefill_kernel<D, CAUSAL, SKIP>;
+  constexpr int smem = PrefillSmem<D>::kDynamic;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const long long grid = p.num_items < sms ? p.num_items : sms;
+  kernel<<<dim3(unsigned(grid)), dim3(kPfThreads), smem, stream>>>(tq, tk, tv, p);
+  return launch_status();
+}
+
+template <int D, bool SKIP>
+int dispatch_prefill_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const PrefillParams& p, int sms, cudaStream_t stream) {
+  return causal ? launch_prefill<D, true, SKIP>(tq, tk, tv, p, sms, stream)
+                : launch_prefill<D, false, SKIP>(tq, tk, tv, p, sms, stream);
+}
+
+int prefill_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S,
+                 int D, int causal, float scale, float lambda, uint8_t* skip_mask, int* device_status,
+                 void* stream, bool blasst) {
+  if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f && lambda < 1.f)) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * S * Hq > (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  int sms = 0;
+  if (int st = current_device(&sms)) return st;
+
+  PrefillParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.skip_mask = skip_mask;
+  p.status = device_status;
+  p.B = B; p.S = S; p.Hq = Hq; p.Hkv = Hkv;
+  p.n_qblocks = (S + 2 * kPfRows - 1) / (2 * kPfRows);
+  p.n_qt = (S + kPfRows - 1) / kPfRows;
+  p.n_kt = (S + 63) / 64;
+  p.num_items = (long long)p.n_qblocks * B * Hq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.log2_lambda = lambda > 0.f ? std::log2(lambda) : -INFINITY;
+
+  CUtensorMap tq, tk, tv;
+  if (int st = encode_bshd(&tq, q, B, S, Hq, D)) return st;
+  if (int st = encode_bshd(&tk, k, B, S, Hkv, D)) return st;
+  if (int st = encode_bshd(&tv, v, B, S, Hkv, D)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool use_skip = blasst && (lambda > 0.f || skip_mask != nullptr);  // the mask needs the decision path
+  if (D == 128)
+    return use_skip ? dispatch_prefill_causal<128, true>(causal != 0, tq, tk, tv, p, sms, s)
+                    : dispatch_prefill_causal<128, false>(causal != 0, tq, tk, tv, p, sms, s);
+  return use_skip ? dispatch_prefill_causal<64, true>(causal != 0, tq, tk, tv, p, sms, s)
+                  : dispatch_prefill_causal<64, false>(causal != 0, tq, tk, tv, p, sms, s);
+}
+
+// ------------------------------------------------------------------ decode
+
+bool valid_page_size(int ps) { return ps == 16 || ps == 32 || ps == 64 || ps == 128 || ps == 256; }
+
+long long max_splits_of(int max_pages, int page_size, int split_tokens) {
+  const long long cap = (long long)max_pages * page_size;
+  return (cap + split_tokens - 1) / split_tokens;
+}
+
+template <int D, int G, bool SKIP>
+int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int sms,
+                  cudaStream_t stream) {
+  auto kernel = decode_split_kernel<D, G, SKIP>;
+  constexpr int smem = DecodeSmem<D, G>::kDynamic;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const long long grid = p.num_items < sms ? p.num_items : sms;
+  kernel<<<dim3(unsigned(grid)), dim3(kDecThreads), smem, stream>>>(tk, tv, p);
+  if (int st = launch_status()) return st;
+  const long long pairs = (long long)p.num_seqs * p.Hq;
+  const long long blocks = (pairs + 7) / 8;
+  decode_merge_kernel<D><<<dim3(unsigned(blocks)), dim3(256), 0, stream>>>(p);
+  return launch_status();
+}
+
+template <int D, bool SKIP>
+int dispatch_decode_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int sms,
+                      cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_decode<D, 1, SKIP>(tk, tv, p, sms, s);
+    case 2: return launch_decode<D, 2, SKIP>(tk, tv, p, sms, s);
+    case 4: return launch_decode<D, 4, SKIP>(tk, tv, p, sms, s);
+    case 8: return launch_decode<D, 8, SKIP>(tk, tv, p, sms, s);
+    case 16: return launch_decode<D, 16, SKIP>(tk, tv, p, sms, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_DEVICE_BOUNDS: return "ATTN_ERR_DEVICE_BOUNDS";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    default: return "ATTN_ERR_UNKNOWN";
+  }
+}
+
+int attn_abi_version(void) { return 1; }
+
+int attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S,
+                 int D, int causal, float scale, void* stream) {
+  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, 0.f, nullptr, nullptr, stream, false);
+}
+
+int attn_prefill_blasst(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int S, int D, int causal, float scale, float lambda, uint8_t* skip_mask,
+                        int* device_status, void* stream) {
+  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, lambda, skip_mask, device_status, stream,
+                      true);
+}
+
+size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq, int page_size,
+                                   int split_tokens) {
+  if (num_seqs < 1 || Hq < 1 || (D != 64 && D != 128) || max_pages_per_seq < 1 || !valid_page_size(page_size) ||
+      split_tokens < 64 || split_tokens % 64 != 0)
+    return 0;
+  const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
+  const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
+  const size_t o_bytes_aligned = (o_bytes + 255) / 256 * 256;
+  return o_bytes_aligned + size_t(num_seqs) * ms * Hq * sizeof(float);
+}
+
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                      const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
+                      int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens, void* o,
+                      float* lse, void* workspace, size_t workspace_bytes, uint8_t* skip_mask, int* device_status,
+                      void* stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace))
+    return ATTN_ERR_INVALID_ARG;
+  if (num_seqs < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!valid_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+  if (split_tokens < 64 || split_tokens % 64 != 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f && lambda < 1.f)) return ATTN_ERR_INVALID_ARG;
+  if ((long long)max_pages_per_seq * page_size > (1ll << 30)) return ATTN_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return ATTN_ERR_UNSUPPORTED;
+  const size_t need = attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens);
+  if (need == 0 || workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
+  int sms = 0;
+  if (int st = current_device(&sms)) return st;
+
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
+  p.ws_o = static_cast<float*>(workspace);
+  const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (o_bytes + 255) / 256 * 256);
+  p.skip_mask = skip_mask;
+  p.status = device_status;
+  p.num_seqs = num_seqs; p.Hq = Hq; p.Hkv = Hkv;
+  p.page_size = page_size; p.max_pages = max_pages_per_seq; p.num_pages = num_pages;
+  p.split_tokens = split_tokens;
+  p.max_splits = int(ms);
+  p.max_tiles = int(((long long)max_pages_per_seq * page_size + 63) / 64);
+  p.chunk = page_size < 64 ? page_size : 64;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.log2_lambda = lambda > 0.f ? std::log2(lambda) : -INFINITY;
+  p.num_items = (long long)num_seqs * ms * Hkv;
+
+  // page pool [P][page_size][Hkv][D] as a 4-D map {D, Hkv, page_size, P}; box = one head of `chunk` tokens
+  const uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(page_size), uint64_t(num_pages)};
+  const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(Hkv) * D * 2, uint64_t(page_size) * Hkv * D * 2};
+  const uint32_t box[4] = {uint32_t(D), 1, uint32_t(p.chunk), 1};
+  CUtensorMap tk, tv;
+  if (int st = encode_map(&tk, k_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return st;
+  if (int st = encode_map(&tv, v_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool use_skip = lambda > 0.f || skip_mask != nullptr;
+  if (D == 128)
+    return use_skip ? dispatch_decode_g<128, true>(G, tk, tv, p, sms, s)
+                    : dispatch_decode_g<128, false>(G, tk, tv, p, sms, s);
+  return use_skip ? dispatch_decode_g<64, true>(G, tk, tv, p, sms, s)
+                  : dispatch_decode_g<64, false>(G, tk, tv, p, sms, s);
+}
+
+int attn_read_device_status(int* status_out, int clear) {
+  if (!status_out) return ATTN_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  *status_out = v;
+  if (clear) {
+    const int zero = ATTN_OK;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,399 @@
+"""Benchmark of the attention hot path on B200.
+
+One step = one causal GQA prefill (B=2, Hq=32, Hkv=8, S=8192, D=128, the shape of
+a Llama-3-8B / Mistral layer) followed by one paged GQA decode (64 sequences,
+lengths uniform in [512, 8192], Hq=32, Hkv=8, D=128, 16-token pages from a
+shared pool in random order). Inputs are seeded synthetic bf16 N(0, 1) data
+resident in HBM. L2 is flushed (a 256 MiB write) before every timed step.
+Kernels are timed with CUDA events on the launching stream.
+
+value = prefill TFLOP/s (algorithmic FLOPs: 4*D per visible (query, key) pair,
+causal diagonal counted exactly); the decode's KV-read GB/s is reported beside
+it. With --gpus N under torchrun every rank runs its own copy of the workload
+(independent problems, weak scaling); times are the max over ranks.
+
+--impl reference times the float64 CPU oracle (test infrastructure) on a
+bounded sample of the same workload, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_online_softmax_fwd_b200 import inputs as gen  # noqa: E402
+
+METRIC = "prefill attn TFLOPS & paged-decode KV-read GB/s, % of B200 roofline"
+PREFILL_CFG = "gqa_prefill_llama3_8b"
+DECODE_CFG = "paged_gqa_decode"
+DECODE_SPLIT = 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def prefill_flops(B, Hq, S, D, causal=True):
+    pairs = S * (S + 1) // 2 if causal else S * S
+    return 4.0 * D * B * Hq * pairs
+
+
+def decode_bytes(seq_lens, Hq, Hkv, D, max_pages):
+    """Algorithmic bytes: every cached K and V row once, plus q, o, lse, tables."""
+    toks = int(sum(seq_lens))
+    n = len(seq_lens)
+    kv = toks * Hkv * D * 2 * 2
+    return kv + n * Hq * D * 2 * 2 + n * Hq * 4 + n * max_pages * 4 + n * 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_profile_traffic():
+    """Per-launch DRAM bytes of the prefill and decode kernels from the committed ncu summary."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f)
+    return {}
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                smax.append(float(parts[2].split()[0]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def dist_max(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(n_prefill_heads=2, n_decode_seqs=4, seed_shift=0):
+    """Time the float64 oracle on a bounded sample of the workload.
+
+    Prefill: ``n_prefill_heads`` (b, hq) heads of the GQA config, all 8192 query
+    rows each. Decode: ``n_decode_seqs`` sequences of the decode config, all
+    query heads. Returns (prefill TFLOP/s, decode GB/s, seconds, description).
+    """
+    from oracle import attn_oracle as orc
+    pc = gen.CONFIGS[PREFILL_CFG]
+    q, k, v = gen.prefill_inputs(1, pc["Hq"], pc["Hkv"], pc["S"], pc["D"], pc["seed"])
+    heads = [(0, (seed_shift * 7 + 5 * i) % pc["Hq"]) for i in range(n_prefill_heads)]
+    t0 = time.perf_counter()
+    orc.prefill(q, k, v, True, gen.attn_scale(pc["D"]), heads=heads)
+    tp = time.perf_counter() - t0
+    fl = prefill_flops(1, len(heads), pc["S"], pc["D"])
+    dc = gen.CONFIGS[DECODE_CFG]
+    cache = gen.paged_decode_inputs(dc["N"], dc["Hq"], dc["Hkv"], dc["D"], dc["page_size"], dc["len_lo"],
+                                    dc["len_hi"], seed=dc["seed"], poison=False)
+    seqs = [(seed_shift * 3 + 9 * i) % dc["N"] for i in range(n_decode_seqs)]
+    t0 = time.perf_counter()
+    orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens,
+                     dc["page_size"], gen.attn_scale(dc["D"]), seqs=seqs)
+    td = time.perf_counter() - t0
+    lens = [int(cache.seq_lens[s]) for s in seqs]
+    by = decode_bytes(lens, dc["Hq"], dc["Hkv"], dc["D"], cache.max_pages)
+    desc = (f"{len(heads)} of {pc['B'] * pc['Hq']} (b,hq) heads of the GQA prefill (all {pc['S']} rows each); "
+            f"{len(seqs)} of {dc['N']} decode sequences")
+    return fl / tp / 1e12, by / td / 1e9, tp + td, desc
+
+
+def cpu_threads():
+    return torch.get_num_threads(), os.cpu_count()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    for i in range(args.warmup):
+        oracle_sample(1, 2, seed_shift=i)
+    tfl, gbs, secs = [], [], 0.0
+    desc = ""
+    for i in range(args.steps):
+        a, b, s, desc = oracle_sample(1, 2, seed_shift=100 + i)
+        tfl.append(a)
+        gbs.append(b)
+        secs += s
+    value = statistics.mean(tfl)
+    cores = cpu_threads()[1]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{PREFILL_CFG}+{DECODE_CFG}", "sample_per_step": desc},
+        "decode": {"value": statistics.mean(gbs), "unit": "GB/s"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, world, rank, local):
+    import attention_online_softmax_fwd_b200 as ab
+    from attention_online_softmax_fwd_b200 import binding
+    binding.load_library()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    pc = gen.CONFIGS[PREFILL_CFG]
+    dc = gen.CONFIGS[DECODE_CFG]
+    B, Hq, Hkv, S, D = pc["B"], pc["Hq"], pc["Hkv"], pc["S"], pc["D"]
+    q_h, k_h, v_h = gen.prefill_inputs(B, Hq, Hkv, S, D, pc["seed"] + 1000 * rank)
+    cache = gen.paged_decode_inputs(dc["N"], dc["Hq"], dc["Hkv"], dc["D"], dc["page_size"], dc["len_lo"],
+                                    dc["len_hi"], seed=dc["seed"] + 1000 * rank, poison=False)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+    dq, dkp, dvp = cache.q.to(dev), cache.k_pages.to(dev), cache.v_pages.to(dev)
+    dbt, dsl = cache.block_table.to(dev), cache.seq_lens.to(dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty((dc["N"], dc["Hq"]), dtype=torch.float32, device=dev)
+    ws = torch.empty(ab.decode_workspace_bytes(dc["N"], dc["Hq"], dc["D"], cache.max_pages, dc["page_size"],
+                                               DECODE_SPLIT), dtype=torch.uint8, device=dev)
+    scale = gen.attn_scale(D)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def prefill_call():
+        ab.prefill(q, k, v, causal=True, scale=scale, out=o, lse=lse)
+
+    def decode_call():
+        ab.decode_paged(dq, dkp, dvp, dbt, dsl, scale=scale, split_tokens=DECODE_SPLIT, out=do, lse=dlse,
+                        workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        prefill_call()
+        decode_call()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        prefill_call()
+        ev[i][1].record(stream)
+        decode_call()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    dec_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    pre_ms = dist_max(pre_ms, world)
+    dec_ms = dist_max(dec_ms, world)
+    step_ms = pre_ms + dec_ms
+
+    # ---- end to end through the public API: pinned host inputs in, results back to host
+    q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    o_p = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
+    lse_p = torch.empty((B, Hq, S), dtype=torch.float32).pin_memory()
+    dq_p, dbt_p, dsl_p = cache.q.pin_memory(), cache.block_table.pin_memory(), cache.seq_lens.pin_memory()
+    do_p = torch.empty(cache.q.shape, dtype=torch.bfloat16).pin_memory()
+    dlse_p = torch.empty((dc["N"], dc["Hq"]), dtype=torch.float32).pin_memory()
+    h2d_pre = sum(t.numel() * t.element_size() for t in (q_p, k_p, v_p))
+    d2h_pre = o_p.numel() * 2 + lse_p.numel() * 4
+    h2d_dec = sum(t.numel() * t.element_size() for t in (dq_p, dbt_p, dsl_p))
+    d2h_dec = do_p.numel() * 2 + dlse_p.numel() * 4
+
+    def e2e_step():
+        q.copy_(q_p, non_blocking=True); k.copy_(k_p, non_blocking=True); v.copy_(v_p, non_blocking=True)
+        prefill_call()
+        o_p.copy_(o, non_blocking=True); lse_p.copy_(lse, non_blocking=True)
+        ee = torch.cuda.Event(enable_timing=True)
+        ee.record(stream)
+        dq.copy_(dq_p, non_blocking=True); dbt.copy_(dbt_p, non_blocking=True); dsl.copy_(dsl_p, non_blocking=True)
+        decode_call()
+        do_p.copy_(do, non_blocking=True); dlse_p.copy_(dlse, non_blocking=True)
+        return ee
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_pre, e2e_dec = [], []
+    for i in range(args.steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e2 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e1 = e2e_step()
+        e2.record(stream)
+        e2.synchronize()
+        e2e_pre.append(e0.elapsed_time(e1))
+        e2e_dec.append(e1.elapsed_time(e2))
+    e2e_pre_ms = dist_max(statistics.mean(e2e_pre), world)
+    e2e_dec_ms = dist_max(statistics.mean(e2e_dec), world)
+
+    # ---- parity spot check of this run's output (cheap invariant: finite, LSE >= row max bound)
+    finite = bool(torch.isfinite(o.float()).all().item() and torch.isfinite(do.float()).all().item())
+
+    peaks, peak_src = load_peaks()
+    traffic = load_profile_traffic()
+    fl = prefill_flops(B, Hq, S, D)
+    by = decode_bytes(cache.seq_lens.tolist(), dc["Hq"], dc["Hkv"], dc["D"], cache.max_pages)
+    pre_tfs = fl / (pre_ms * 1e-3) / 1e12
+    dec_gbs = by / (dec_ms * 1e-3) / 1e9
+    value = pre_tfs * world
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{PREFILL_CFG}+{DECODE_CFG}",
+            "prefill": {"B": B, "Hq": Hq, "Hkv": Hkv, "S": S, "D": D, "causal": True, "seed": pc["seed"]},
+            "decode": {"num_seqs": dc["N"], "Hq": dc["Hq"], "Hkv": dc["Hkv"], "D": dc["D"],
+                       "page_size": dc["page_size"], "len_range": [dc["len_lo"], dc["len_hi"]],
+                       "split_tokens": DECODE_SPLIT, "tokens": int(cache.seq_lens.sum()), "seed": dc["seed"]},
+            "l2": "flushed before every timed step (256 MiB write)",
+            "parallelism": f"replica x{world}" if world > 1 else "single GPU",
+        },
+        "prefill": {"ms": pre_ms, "tflops": pre_tfs, "flops_per_launch": fl,
+                    "frac_of_spec_2250": pre_tfs / SPEC_PEAKS["bf16_tflops"]},
+        "decode": {"ms": dec_ms, "value": dec_gbs * world, "unit": "GB/s", "bytes_per_call": by,
+                   "frac_of_spec_8000": dec_gbs / SPEC_PEAKS["hbm_gbs"]},
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel<128,causal>", "achieved": pre_tfs,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": pre_tfs / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16 burst", "traffic": traffic.get("prefill_bytes_per_launch")},
+        "roofline_decode": {"bound": "hbm", "kernel": "decode_split_kernel<128,4>+decode_merge_kernel",
+                            "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": dec_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy",
+                            "traffic": traffic.get("decode_bytes_per_call")},
+        "e2e": {"value": fl / (e2e_pre_ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d_pre + h2d_dec, "d2h_bytes_per_step": d2h_pre + d2h_dec,
+                "prefill_ms": e2e_pre_ms, "decode_ms": e2e_dec_ms,
+                "decode_gbs": by / (e2e_dec_ms * 1e-3) / 1e9 * world},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+        "wall_s_timed_region": wall,
+        "outputs_finite": finite,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tfs, gbs, secs, desc = oracle_sample(int(args.cpu_heads), 4)
+        line["cpu_baseline"] = {"value": tfs, "unit": "TFLOP/s", "cores": cpu_threads()[0], "kind": "oracle",
+                                "sample": desc, "decode_gbs": gbs, "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=8)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

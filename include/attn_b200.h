@@ -1,0 +1,165 @@
+/*
+ * attn_b200.h -- C ABI of the B200 (sm_100a) exact-attention forward library.
+ *
+ * Two operations, each an exact scaled-dot-product attention forward with an
+ * online (blockwise, running-maximum) softmax:
+ *
+ *   prefill  O = softmax(Q K^T * scale + causal mask) V over whole sequences,
+ *            tiled so that no S x S matrix ever reaches global memory
+ *            ("flash-attention与TensorRT-LLM集成", section FlashAttention工作原理:
+ *            Q/K/V are split into blocks that are loaded and released on the fly
+ *            and memory stays linear in S; "LLM推理优化技术综述", PART04).
+ *   decode   one new query token per sequence against its cached keys and
+ *            values, which live in fixed-size pages of a shared pool addressed
+ *            through a per-sequence block table ("LLM推理优化技术综述", PART02;
+ *            "Optimizing Inference on LLMs with TensorRT-LLM", PagedAttention;
+ *            "TensorRT对Grouped Query Attention的支持进展", 动态形状与KV Cache管理:
+ *            the caller hands in physical page indices every decode step).
+ *
+ * Grouped-query attention: query head h reads KV head h / (Hq / Hkv)
+ * ("TensorRT对Grouped Query Attention的支持进展", 技术演进背景; "LLM推理优化技术综述",
+ * PART03). Hkv == Hq is MHA, Hkv == 1 is MQA.
+ *
+ * Optional BLASST tile skip ("高效部署稀疏注意力加速方案：BLASST方法详解与实践指南",
+ * 架构与组件): with lambda > 0, a tile of 64 keys is skipped -- no exponentials,
+ * no V load, no P V product -- when exp(tile_rowmax - running_max) < lambda for
+ * every row of its decision unit. The running maximum is over the unit's tiles
+ * already kept, in ascending key order. lambda == 0 computes the dense result.
+ *
+ * Common conventions
+ *   - Every pointer is a DEVICE pointer owned by the caller. The library never
+ *     allocates, frees or synchronises; all work is enqueued on `stream`
+ *     (a cudaStream_t; NULL is the legacy default stream).
+ *   - bf16 means IEEE bfloat16 (__nv_bfloat16), row-major, contiguous.
+ *     Accumulation is fp32. LSE is the natural-log log-sum-exp of the scaled
+ *     scores, fp32.
+ *   - q/k/v/o/page pointers must be 16-byte aligned.
+ *   - Head dimension D must be 64 or 128.
+ *   - Return value: ATTN_OK, or an error code. Argument errors are detected on
+ *     the host before anything is enqueued. Errors found on the device
+ *     (out-of-range block-table entries, a pipeline wait that timed out) are
+ *     reported through `device_status` when given, and always through the
+ *     library's device status word (attn_read_device_status). No kernel traps.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or lambda        */
+  ATTN_ERR_UNSUPPORTED = 2,   /* device is not sm_100, or an unsupported shape */
+  ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed   */
+  ATTN_ERR_DEVICE_BOUNDS = 4, /* a block_table entry was outside [0, pages)    */
+  ATTN_ERR_TIMEOUT = 5        /* a kernel pipeline wait expired; output invalid */
+};
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* attn_status_string(int status);
+
+/* ABI version, bumped on any incompatible change. */
+int attn_abi_version(void);
+
+/*
+ * attn_prefill -- dense causal or non-causal prefill attention.
+ *
+ *   q    [B][S][Hq][D]  bf16     queries
+ *   k, v [B][S][Hkv][D] bf16     keys and values (key j of a sequence is token j)
+ *   o    [B][S][Hq][D]  bf16     output, written completely
+ *   lse  [B][Hq][S]     fp32     log-sum-exp per query row; may be NULL
+ *   causal != 0: key j is visible to query i iff j <= i
+ *   scale: multiplies Q K^T (typically 1/sqrt(D))
+ * Requirements: B >= 1, S >= 1, Hkv >= 1, Hq % Hkv == 0, D in {64, 128}.
+ * Work is (b, hq, 128-row query tile); every pair of query rows sees exactly
+ * the keys the definition lets it see; ragged S is handled inside the kernel.
+ */
+int attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int S, int D, int causal, float scale,
+                 void* stream);
+
+/*
+ * attn_prefill_blasst -- attn_prefill with the BLASST tile skip.
+ *
+ * Decision unit: (b, hq, query tile of rows [128 t, min(128 t + 128, S))).
+ * Its tiles are the 64-key tiles in ascending order (causal: only tiles whose
+ * first key is <= the unit's last row). lambda in [0, 1).
+ *   skip_mask  [B][Hq][ceil(S/128)][ceil(S/64)] uint8, may be NULL. For every
+ *              visited tile the kernel writes 1 (skipped) or 0 (kept); entries
+ *              of tiles never visited are left untouched.
+ *   device_status  int on the device, may be NULL; set (never cleared) to a
+ *              device-side error code.
+ * The output and LSE are those of attention restricted to the kept keys.
+ */
+int attn_prefill_blasst(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int Hq, int Hkv, int S, int D, int causal, float scale,
+                        float lambda, uint8_t* skip_mask, int* device_status,
+                        void* stream);
+
+/*
+ * attn_decode_workspace_bytes -- scratch needed by attn_decode_paged.
+ * The decode splits each sequence's keys into chunks of split_tokens tokens,
+ * computes one partial (O, LSE) per (sequence, query head, chunk), and merges
+ * them. The workspace holds those partials:
+ *   fp32 [num_seqs][max_splits][Hq][D] + fp32 [num_seqs][max_splits][Hq]
+ * with max_splits = ceil(max_pages_per_seq * page_size / split_tokens).
+ * Returns 0 for invalid arguments.
+ */
+size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq,
+                                   int page_size, int split_tokens);
+
+/*
+ * attn_decode_paged -- single-token decode over a paged KV cache (split-KV
+ * kernel followed by a log-sum-exp merge kernel).
+ *
+ *   q            [num_seqs][Hq][D] bf16          one query token per sequence
+ *   k_pages,
+ *   v_pages      [num_pages][page_size][Hkv][D] bf16   the shared page pool
+ *   block_table  [num_seqs][max_pages_per_seq] int32   physical page of each
+ *                logical page; entries past the last used page are ignored
+ *   seq_lens     [num_seqs] int32 (device)       cached tokens per sequence;
+ *                the query sees tokens [0, seq_len). 0 gives o = 0, lse = -inf.
+ *                Must be <= max_pages_per_seq * page_size (checked on the
+ *                device: excess tokens are dropped and ATTN_ERR_DEVICE_BOUNDS set).
+ *   page_size    16, 32, 64, 128 or 256 tokens
+ *   lambda       0 for dense; in (0, 1) for the BLASST skip, whose decision
+ *                unit is (sequence, KV head, split): the rows are the
+ *                Hq / Hkv query heads sharing the KV head, the tiles the split's
+ *                64-token tiles, the running maximum restarts at each split
+ *   split_tokens multiple of 64 (>= 64): tokens per split
+ *   o            [num_seqs][Hq][D] bf16, lse [num_seqs][Hq] fp32 (lse may be NULL)
+ *   workspace    device scratch of at least attn_decode_workspace_bytes(...)
+ *                bytes, 16-byte aligned; contents on entry are ignored
+ *   skip_mask    [num_seqs][Hkv][ceil(max_pages_per_seq*page_size/64)] uint8,
+ *                may be NULL: 1 skipped / 0 kept for every visited tile; other
+ *                entries untouched
+ *   device_status  may be NULL (see attn_prefill_blasst)
+ * A block_table entry outside [0, num_pages) is never dereferenced: its
+ * tokens are treated as absent and ATTN_ERR_DEVICE_BOUNDS is raised.
+ * Hq / Hkv must be 1, 2, 4, 8 or 16.
+ */
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                      const int32_t* block_table, const int32_t* seq_lens,
+                      int num_seqs, int Hq, int Hkv, int D, int page_size,
+                      int max_pages_per_seq, int num_pages, float scale, float lambda,
+                      int split_tokens, void* o, float* lse,
+                      void* workspace, size_t workspace_bytes,
+                      uint8_t* skip_mask, int* device_status, void* stream);
+
+/*
+ * attn_read_device_status -- read (and, if clear != 0, reset to ATTN_OK) the
+ * library's device status word on the current device. Synchronises the
+ * device. Every kernel of the library ORs a device-side error into it.
+ */
+int attn_read_device_status(int* status_out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

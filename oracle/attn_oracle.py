@@ -127,18 +127,21 @@ def prefill(q, k, v, causal: bool, scale: float, row_block: int = 2048,
 
 
 def gather_pages(pages, block_table_row, seq_len: int, page_size: int):
-    """Contiguous [seq_len, Hkv, D] view of one sequence's paged K or V.
+    """Contiguous [seq_len, Hkv, D] float64 view of one sequence's paged K or V.
 
     pages [P, page_size, Hkv, D]; token p is pages[block_table_row[p // page_size], p % page_size].
+    Only the pages the sequence uses are read (and widened).
     """
-    pages = _f64(pages)
-    out = np.empty((seq_len,) + pages.shape[2:])
-    for p in range(seq_len):
-        page = int(block_table_row[p // page_size])
-        if page < 0 or page >= pages.shape[0]:
-            raise IndexError(f"block_table entry {page} out of range for token {p}")
-        out[p] = pages[page, p % page_size]
-    return out
+    n_pages = -(-seq_len // page_size)
+    ids = [int(x) for x in block_table_row[:n_pages]]
+    n_pool = pages.shape[0]
+    for j, page in enumerate(ids):
+        if page < 0 or page >= n_pool:
+            raise IndexError(f"block_table entry {page} out of range for logical page {j}")
+    if n_pages == 0:
+        return np.empty((0,) + tuple(pages.shape[2:]))
+    picked = _f64(pages[ids])                           # [n_pages, page_size, Hkv, D]
+    return picked.reshape((n_pages * page_size,) + picked.shape[2:])[:seq_len]
 
 
 def decode_paged(q, k_pages, v_pages, block_table, seq_lens, page_size: int, scale: float,

@@ -1,0 +1,123 @@
+"""The C ABI library loads, exports what the header declares, and validates on the host.
+
+These run without a GPU: every call here is rejected by host-side checks
+before any CUDA work is enqueued (or fails with ATTN_ERR_CUDA when no device
+is present), so no kernel is launched.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_online_softmax_fwd_b200 as ab
+from attention_online_softmax_fwd_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+
+OK, INVALID, UNSUPPORTED, CUDA = 0, 1, 2, 3
+FAKE = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced on the host
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def test_header_and_binding_agree(lib):
+    names = declared_functions()
+    assert "attn_prefill" in names and "attn_decode_paged" in names
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in the header but not exported"
+        assert name in binding.SIGNATURES, f"{name} has no binding signature"
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        assert lib.attn_status_string(code).decode() == name
+    assert lib.attn_status_string(99).decode() == "ATTN_ERR_UNKNOWN"
+    assert lib.attn_abi_version() == 1
+
+
+def _prefill(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=4, Hkv=2, S=128, D=64, causal=1, scale=0.125)
+    a.update(kw)
+    return lib.attn_prefill(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["S"],
+                            a["D"], a["causal"], a["scale"], None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(o=None), dict(q=ctypes.c_void_p((1 << 20) + 8)),
+                                 dict(B=0), dict(S=0), dict(Hq=3), dict(Hkv=0), dict(scale=0.0),
+                                 dict(scale=float("nan")), dict(scale=-1.0)])
+def test_prefill_rejects_bad_arguments(lib, bad):
+    assert _prefill(lib, **bad) == INVALID
+
+
+def test_prefill_rejects_unsupported_head_dim(lib):
+    assert _prefill(lib, D=96) == UNSUPPORTED
+
+
+def test_prefill_blasst_rejects_bad_lambda(lib):
+    for lam in (-0.1, 1.0, 2.0, float("nan")):
+        st = lib.attn_prefill_blasst(FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, 64, 1, 0.125, lam, None, None,
+                                     None)
+        assert st == INVALID
+
+
+def test_workspace_bytes(lib):
+    # fp32 [N][splits][Hq][D] padded to 256 B, then fp32 [N][splits][Hq]
+    n, hq, d, mp, ps, sp = 64, 32, 128, 512, 16, 1024
+    splits = -(-mp * ps // sp)
+    o_bytes = n * splits * hq * d * 4
+    want = -(-o_bytes // 256) * 256 + n * splits * hq * 4
+    assert lib.attn_decode_workspace_bytes(n, hq, d, mp, ps, sp) == want
+    assert ab.decode_workspace_bytes(n, hq, d, mp, ps, sp) == want
+    for bad in [(0, hq, d, mp, ps, sp), (n, hq, 96, mp, ps, sp), (n, hq, d, mp, 24, sp), (n, hq, d, mp, ps, 100),
+                (n, hq, d, 0, ps, sp)]:
+        assert lib.attn_decode_workspace_bytes(*bad) == 0
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, N=4, Hq=8, Hkv=2, D=128, ps=16, mp=8, P=64,
+             scale=0.09, lam=0.0, split=64, o=FAKE, lse=None, ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    return lib.attn_decode_paged(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["N"], a["Hq"], a["Hkv"], a["D"],
+                                 a["ps"], a["mp"], a["P"], a["scale"], a["lam"], a["split"], a["o"], a["lse"],
+                                 a["ws"], a["wsb"], None, None, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(bt=None), dict(sl=None), dict(ws=None), dict(N=0),
+                                 dict(Hq=6, Hkv=4), dict(ps=24), dict(ps=0), dict(split=96), dict(split=0),
+                                 dict(mp=0), dict(P=0), dict(lam=1.0), dict(lam=-0.5), dict(wsb=16),
+                                 dict(kp=ctypes.c_void_p((1 << 20) + 4))])
+def test_decode_rejects_bad_arguments(lib, bad):
+    assert _decode(lib, **bad) == INVALID
+
+
+@pytest.mark.parametrize("bad", [dict(D=80), dict(Hq=24, Hkv=1), dict(Hq=6, Hkv=2)])
+def test_decode_rejects_unsupported(lib, bad):
+    assert _decode(lib, **bad) == UNSUPPORTED
+
+
+def test_valid_arguments_without_a_device_report_cuda_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert _prefill(lib) == CUDA
+    assert _decode(lib) == CUDA
+
+
+def test_binding_fails_loudly_when_library_missing(monkeypatch):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "lib_path", lambda: "/nonexistent/libattn_b200.so")
+    with pytest.raises(binding.AttnError):
+        binding.load_library()

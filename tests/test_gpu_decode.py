@@ -1,0 +1,106 @@
+"""Paged decode on the GPU, through the C ABI, against the float64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import attention_online_softmax_fwd_b200 as ab
+from attention_online_softmax_fwd_b200 import inputs as gen
+from oracle import attn_oracle as orc
+from parity_util import compare_output, compare_skip
+
+pytestmark = pytest.mark.gpu
+
+
+def _to(cache, dev):
+    return [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+
+
+def _run(cache, dev, split, lam=None):
+    q, kp, vp, bt, sl = _to(cache, dev)
+    scale = gen.attn_scale(q.shape[-1])
+    if lam is None:
+        o, lse = ab.decode_paged(q, kp, vp, bt, sl, scale=scale, split_tokens=split)
+        mask = None
+    else:
+        o, lse, mask = ab.decode_paged_blasst(q, kp, vp, bt, sl, lam, scale=scale, split_tokens=split)
+    torch.cuda.synchronize()
+    return o, lse, mask, scale
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 2, 128), (8, 8, 64), (16, 1, 128), (4, 2, 64), (32, 16, 128),
+                                      (16, 2, 128)])
+@pytest.mark.parametrize("page_size", [16, 64, 256])
+def test_decode_small(cuda_device, Hq, Hkv, D, page_size):
+    lens = [1, 63, 64, 65, 700, 2049, 0, 130]
+    cache = gen.paged_decode_inputs(len(lens), Hq, Hkv, D, page_size, 0, 0, seed=2000 + Hq + D + page_size,
+                                    lens=lens)
+    for split in (64, 128, 1024):
+        o, lse, _, scale = _run(cache, cuda_device, split)
+        o_ref, lse_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table,
+                                          cache.seq_lens, page_size, scale)
+        o_ref[6], lse_ref[6] = 0.0, -np.inf
+        compare_output(o, o_ref, lse, lse_ref, label=f"decode split={split}")
+
+
+def test_decode_paged_gqa_full_size(cuda_device):
+    """64 sequences, lengths uniform in [512, 8192], Hq=32, Hkv=8, D=128, page 16, split 1024."""
+    c = gen.CONFIGS["paged_gqa_decode"]
+    cache = gen.paged_decode_inputs(c["N"], c["Hq"], c["Hkv"], c["D"], c["page_size"], c["len_lo"], c["len_hi"],
+                                    seed=c["seed"])
+    o, lse, _, scale = _run(cache, cuda_device, 1024)
+    o_ref, lse_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens,
+                                      c["page_size"], scale)
+    stats = compare_output(o, o_ref, lse, lse_ref, label="paged_gqa_decode")
+    print("paged_gqa_decode", stats)
+
+
+def test_decode_deterministic(cuda_device):
+    cache = gen.paged_decode_inputs(16, 32, 8, 128, 16, 100, 3000, seed=2100)
+    o1, l1, _, _ = _run(cache, cuda_device, 256)
+    o2, l2, _, _ = _run(cache, cuda_device, 256)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("split", [256, 2048])
+@pytest.mark.parametrize("lam", [0.1, 0.3])
+def test_decode_blasst_matches_oracle(cuda_device, split, lam):
+    S, Hq, Hkv, D = 4096, 32, 8, 128
+    q, k, v = gen.peaked_prefill_inputs(1, Hq, Hkv, S, D, seed=2200, amp=4.0)
+    cache = gen.paged_from_contiguous(q[:, S - 1], k, v, page_size=16, seed=2201)
+    o, lse, mask, scale = _run(cache, cuda_device, split, lam)
+    o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages,
+                                                            cache.block_table, cache.seq_lens, 16, scale, lam,
+                                                            split)
+    st = compare_skip(mask, m_ref, margin, label=f"decode skip lam={lam}")
+    assert st["skipped"] > 0
+    if st["tie_mismatches"] == 0:
+        compare_output(o, o_ref, lse, lse_ref, label=f"decode blasst lam={lam}")
+
+
+def test_decode_lambda_zero_mask_is_dense(cuda_device):
+    cache = gen.paged_decode_inputs(8, 32, 8, 128, 16, 64, 2000, seed=2300)
+    o0, l0, _, scale = _run(cache, cuda_device, 512)
+    o1, l1, mask, _ = _run(cache, cuda_device, 512, 0.0)
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    _, _, m_ref, margin = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages, cache.block_table,
+                                                  cache.seq_lens, 16, scale, 0.0, 512)
+    compare_skip(mask, m_ref, margin)
+    assert not (mask == 1).any()
+
+
+def test_decode_bad_page_raises_device_status(cuda_device):
+    cache = gen.paged_decode_inputs(4, 8, 2, 128, 16, 100, 300, seed=2400)
+    cache.block_table[1, 2] = cache.num_pages + 5      # out of range: never dereferenced
+    cache.block_table[2, 0] = -7
+    q, kp, vp, bt, sl = _to(cache, cuda_device)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ab.binding.read_device_status(clear=True)
+    o, lse = ab.decode_paged(q, kp, vp, bt, sl, split_tokens=64, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 4                        # ATTN_ERR_DEVICE_BOUNDS
+    assert ab.binding.read_device_status(clear=True) == 4
+    # sequences with valid tables are unaffected
+    o_ref, lse_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens,
+                                      16, gen.attn_scale(128), seqs=[0, 3])
+    compare_output(o[[0, 3]], o_ref[[0, 3]], lse[[0, 3]], lse_ref[[0, 3]])
