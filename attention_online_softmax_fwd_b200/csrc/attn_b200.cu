@@ -269,13 +269,14 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   p.log2_lambda = lambda > 0.f ? std::log2(lambda) : -INFINITY;
   p.num_items = (long long)num_seqs * ms * Hkv;
 
-  // page pool [P][page_size][Hkv][D] as a 4-D map {D, Hkv, page_size, P}; box = one head of `chunk` tokens
+  // page pool [P][page_size][Hkv][D] as a 4-D map {D, Hkv, page_size, P}; box = 64 columns of one head
+  // for `chunk` tokens, written with the 128-byte swizzle
   const uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(page_size), uint64_t(num_pages)};
   const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(Hkv) * D * 2, uint64_t(page_size) * Hkv * D * 2};
-  const uint32_t box[4] = {uint32_t(D), 1, uint32_t(p.chunk), 1};
+  const uint32_t box[4] = {64, 1, uint32_t(p.chunk), 1};
   CUtensorMap tk, tv;
-  if (int st = encode_map(&tk, k_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return st;
-  if (int st = encode_map(&tv, v_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return st;
+  if (int st = encode_map(&tk, k_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return st;
+  if (int st = encode_map(&tv, v_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool use_skip = lambda > 0.f || skip_mask != nullptr;
   if (D == 128)

@@ -2,15 +2,23 @@
 //
 // Work item = (sequence, split, KV head). A persistent CTA walks its items in
 // a strided order. One producer warp streams the item's 64-token tiles of K
-// and V from the page pool into a shared-memory ring with TMA copies, one copy
-// per (page chunk, K|V), addressed through the block table. Eight consumer
-// warps each take 8 tokens of a tile and all G query heads of the KV head:
-// lanes split the head dimension for q.k (partial dots reduced with a
-// butterfly reduce-scatter) and for P.V. The softmax state (running max m,
-// sum l, accumulator O) follows the online recurrence over the split's tiles;
-// m is shared by the eight warps (one named barrier per tile), l and O are
-// per warp and summed at the end of the item. A split's result is written as a
-// partial (O / l, log2-sum-exp); the merge kernel combines the splits.
+// and V from the page pool into a shared-memory ring with TMA, one copy per
+// (page chunk, 64-column half, K|V), addressed through the block table. The
+// copies use the 128-byte swizzle so that the consumers' ldmatrix reads are
+// free of bank conflicts.
+//
+// Four consumer warps each take 16 tokens of a tile. The G query heads that
+// share the KV head are the rows of a 16-row operand (rows >= G are zero), so
+// q.K^T and P.V are two small matrix products per tile, done with
+// mma.m16n8k16 (bf16 in, fp32 accumulate, in registers). The online softmax
+// (running reference maximum, sum, accumulator) runs per warp in the
+// accumulator registers; the four warps' states are merged in a fixed order
+// at the end of the item. With the tile skip enabled, the warps exchange
+// their tile maxima once per tile (one named barrier) so that every warp sees
+// the tile's true row maxima and the unit's true running maximum.
+// A split's result is written as a partial (O / l, log2-sum-exp); the merge
+// kernel combines the splits of a sequence. A sequence with one split is
+// written directly by the split kernel.
 #pragma once
 
 #include "common.cuh"
@@ -36,24 +44,26 @@ struct DecodeParams {
 };
 
 constexpr int kDecTile = 64;          // tokens per tile (= BLASST decision tile)
-constexpr int kDecConsumerWarps = 8;  // 8 tokens of each tile per warp
+constexpr int kDecConsumerWarps = 4;  // 16 tokens of each tile per warp
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
-constexpr int kDecStages = 4;
+constexpr float kDecRescaleThreshold = 8.0f;  // log2 units
 
 template <int D, int G>
 struct DecodeSmem {
-  static constexpr int kStageBytes = 2 * kDecTile * D * 2;  // K and V tiles, bf16
-  static constexpr int kRing = kDecStages * kStageBytes;
-  // offsets (bytes) from the 1024-aligned base
-  static constexpr int kFull = kRing;
-  static constexpr int kEmpty = kFull + 8 * kDecStages;
-  static constexpr int kInfo = kEmpty + 8 * kDecStages;                  // int2 per stage
-  static constexpr int kScore = kInfo + 8 * kDecStages;                  // [warps][8*G] floats
-  static constexpr int kRed = kScore + 4 * kDecConsumerWarps * 8 * G;    // [2][warps][G] floats
-  static constexpr int kCombL = kRed + 4 * 2 * kDecConsumerWarps * G;    // [2][G] floats
-  static constexpr int kCombO = (kCombL + 4 * 2 * G + 15) / 16 * 16;     // [G][D] floats
-  static constexpr int kTotal = kCombO + 4 * G * D;
-  static constexpr int kDynamic = kTotal + 1024;                         // slack for alignment
+  static constexpr int kHalfBytes = kDecTile * 128;            // 64 tokens x 64 columns, 128B-swizzled
+  static constexpr int kTileBytes = kDecTile * D * 2;          // one K or V tile
+  static constexpr int kStageBytes = 2 * kTileBytes;           // K then V
+  static constexpr int kStages = D == 128 ? 6 : 12;
+  static constexpr int kRing = kStages * kStageBytes;
+  static constexpr int kFull = kRing;                                   // mbarriers
+  static constexpr int kEmpty = kFull + 8 * kStages;
+  static constexpr int kInfo = kEmpty + 8 * kStages;                    // int2 per stage
+  static constexpr int kRed = kInfo + 8 * kStages;                      // [2][warps][16] floats
+  static constexpr int kCombM = kRed + 4 * 2 * kDecConsumerWarps * 16;  // [warps][G] floats
+  static constexpr int kCombL = kCombM + 4 * kDecConsumerWarps * G;     // [warps][G] floats
+  static constexpr int kCombO = (kCombL + 4 * kDecConsumerWarps * G + 15) / 16 * 16;  // [warps][G][D]
+  static constexpr int kTotal = kCombO + 4 * kDecConsumerWarps * G * D;
+  static constexpr int kDynamic = kTotal + 1024;                        // slack for alignment
 };
 
 __device__ __forceinline__ void decode_item_coords(long long item, int Hkv, int max_splits, int& seq, int& split,
@@ -64,37 +74,28 @@ __device__ __forceinline__ void decode_item_coords(long long item, int Hkv, int 
   seq = int(rest / max_splits);
 }
 
-// Load the D/32 consecutive bf16 of one row that belong to `lane`, as fp32.
-template <int D>
-__device__ __forceinline__ void load_row_slice(const __nv_bfloat16* row, int lane, float (&x)[D / 32]) {
-  if constexpr (D == 128) {
-    const uint2 w = *reinterpret_cast<const uint2*>(row + lane * 4);
-    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-  } else {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(row + lane * 2);
-    x[0] = bf16_lo(w); x[1] = bf16_hi(w);
-  }
+// Byte offset of 16-byte chunk `c` (0 .. D/8-1) of token row `r` in a swizzled tile.
+__device__ __forceinline__ uint32_t swz_off(int r, int c) {
+  return uint32_t((c >> 3) * (kDecTile * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
 template <int D, int G, bool SKIP>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeParams p) {
+  static_assert(G >= 1 && G <= 16, "query heads per KV head");
   using L = DecodeSmem<D, G>;
-  constexpr int DL = D / 32;                              // head dims per lane
-  constexpr int TB = (G >= 4) ? (32 / G < 1 ? 1 : 32 / G) : 8;  // tokens per reduce batch
-  constexpr int TBc = TB > 8 ? 8 : TB;
-  constexpr int NB = 8 / TBc;                             // reduce batches per tile
-  constexpr int V = TBc * G;                              // values per batch (<= 32)
-  constexpr int DUP = 32 / V;                             // lanes holding the same value
+  constexpr int NS = L::kStages;
+  constexpr int KS = D / 16;   // k-steps of q.K^T
+  constexpr int NT = D / 8;    // 8-column tiles of O
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kFull);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::kEmpty);
   int2* info = reinterpret_cast<int2*>(smem + L::kInfo);
-  float* score = reinterpret_cast<float*>(smem + L::kScore);
   float* red = reinterpret_cast<float*>(smem + L::kRed);
+  float* comb_m = reinterpret_cast<float*>(smem + L::kCombM);
   float* comb_l = reinterpret_cast<float*>(smem + L::kCombL);
   float* comb_o = reinterpret_cast<float*>(smem + L::kCombO);
   __shared__ int abort_flag;
@@ -105,14 +106,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int s = 0; s < kDecStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kDecConsumerWarps);
     }
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) comb_o[i] = 0.f;
-  for (int i = threadIdx.x; i < 2 * G; i += blockDim.x) comb_l[i] = 0.f;
   __syncthreads();
 
   if (warp == kDecConsumerWarps) {
@@ -122,7 +121,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tma_prefetch_desc(&tm_v);
     }
     const int nchunks = kDecTile / p.chunk;
-    const uint32_t chunk_bytes = uint32_t(p.chunk) * D * 2;
+    const uint32_t chunk_bytes = uint32_t(p.chunk) * D * 2;   // one K (or V) chunk, both halves
     int slot = 0;
     uint32_t phase = 0;
     uint32_t pending = 0;  // stages with copies issued, for the abort path
@@ -140,19 +139,34 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (t_begin >= len) continue;
       const int t_end = min(t_begin + p.split_tokens, len);
       const int32_t* bt_row = p.block_table + size_t(seq) * p.max_pages;
+      // Block-table entries are fetched 32 at a time (one per lane), one window
+      // ahead, so that a tile's page ids are a shuffle away when it is issued.
+      const int n_entries = (len + p.page_size - 1) / p.page_size;
+      auto load_window = [&](int w) {
+        const int e = w * 32 + lane;
+        return e < n_entries ? __ldg(&bt_row[e]) : -1;
+      };
+      int win = (t_begin / p.page_size) >> 5;
+      int win_cur = load_window(win);
+      int win_next = load_window(win + 1);
       for (int t0 = t_begin; t0 < t_end; t0 += kDecTile) {
+        const int e0 = t0 / p.page_size;  // first entry of this tile; a tile never straddles a window
+        if ((e0 >> 5) != win) {
+          win = e0 >> 5;
+          win_cur = win_next;
+          win_next = load_window(win + 1);
+        }
         if (!mbar_wait(&empty[slot], phase ^ 1u, &abort_flag, p.status)) { ok = false; break; }
-        int page = -1;
+        const int p0 = t0 + lane * p.chunk;
+        const int mine =
+            __shfl_sync(0xffffffffu, win_cur, (e0 & 31) + (lane < nchunks ? lane * p.chunk / p.page_size : 0));
+        int page = -1, in_page = 0;
         bool valid = false, bad = false;
-        int in_page = 0;
-        if (lane < nchunks) {
-          const int p0 = t0 + lane * p.chunk;
-          if (p0 < len) {
-            page = __ldg(&bt_row[p0 / p.page_size]);
-            in_page = p0 % p.page_size;
-            valid = page >= 0 && page < p.num_pages;
-            bad = !valid;
-          }
+        if (lane < nchunks && p0 < len) {
+          page = mine;
+          in_page = p0 % p.page_size;
+          valid = page >= 0 && page < p.num_pages;
+          bad = !valid;
         }
         const uint32_t valid_mask = __ballot_sync(0xffffffffu, valid);
         const uint32_t bad_mask = __ballot_sync(0xffffffffu, bad);
@@ -163,29 +177,38 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         __syncwarp();
         if (valid) {
-          uint8_t* kdst = smem + slot * L::kStageBytes + lane * chunk_bytes;
-          uint8_t* vdst = kdst + kDecTile * D * 2;
-          tma_load_4d(kdst, &tm_k, &full[slot], 0, kvh, in_page, page);
-          tma_load_4d(vdst, &tm_v, &full[slot], 0, kvh, in_page, page);
+          uint8_t* kbase = smem + slot * L::kStageBytes;
+          uint8_t* vbase = kbase + L::kTileBytes;
+          const int row0 = lane * p.chunk;
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            tma_load_4d(kbase + h * L::kHalfBytes + row0 * 128, &tm_k, &full[slot], h * 64, kvh, in_page, page);
+            tma_load_4d(vbase + h * L::kHalfBytes + row0 * 128, &tm_v, &full[slot], h * 64, kvh, in_page, page);
+          }
         }
         pending |= 1u << slot;
         pending_phase = (pending_phase & ~(1u << slot)) | (phase << slot);
-        if (++slot == kDecStages) { slot = 0; phase ^= 1u; }
+        if (++slot == NS) { slot = 0; phase ^= 1u; }
       }
     }
     if (!ok && lane == 0) {
-      for (int s = 0; s < kDecStages; ++s)
+      for (int s = 0; s < NS; ++s)
         if (pending & (1u << s)) mbar_drain(&full[s], (pending_phase >> s) & 1u);
     }
   } else {
     // ------------------------------------------------------------ consumer warps
+    const float neg_inf = -__int_as_float(0x7f800000);
+    const int g = lane >> 2;         // accumulator row (query head within the group)
+    const int tq = lane & 3;         // column pair within an 8-column tile
+    const bool row0_valid = g < G;   // rows g and g + 8
+    const bool row1_valid = g + 8 < G;
     int slot = 0;
     uint32_t phase = 0;
     int red_par = 0;
-    int item_par = 0;
     int no_abort = 0;  // consumers stop only on their own timeout (see mbar_wait)
     bool ok = true;
-    const float neg_inf = -__int_as_float(0x7f800000);
+    const uint32_t ring_addr = smem_u32(smem);
+
     for (long long item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
       int seq, split, kvh;
       decode_item_coords(item, p.Hkv, p.max_splits, seq, split, kvh);
@@ -196,25 +219,28 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int t_end = min(t_begin + p.split_tokens, len);
       const int n_splits = (len + p.split_tokens - 1) / p.split_tokens;
 
-      // q for the G heads of this KV head, pre-scaled into the log2 domain
-      float qf[G][DL];
+      // q of the G heads as the A operand (rows >= G are zero)
+      uint32_t qa[KS][4];
+      {
+        const int h0 = row0_valid ? g : 0, h1 = row1_valid ? g + 8 : 0;
+        const uint32_t* q0 =
+            reinterpret_cast<const uint32_t*>(p.q + (size_t(seq) * p.Hq + size_t(kvh) * G + h0) * D);
+        const uint32_t* q1 =
+            reinterpret_cast<const uint32_t*>(p.q + (size_t(seq) * p.Hq + size_t(kvh) * G + h1) * D);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const __nv_bfloat16* qrow = p.q + (size_t(seq) * p.Hq + size_t(kvh) * G + h) * D;
-        float x[DL];
-        load_row_slice<D>(qrow, lane, x);
-#pragma unroll
-        for (int d = 0; d < DL; ++d) qf[h][d] = x[d] * p.scale_log2;
+        for (int ks = 0; ks < KS; ++ks) {
+          qa[ks][0] = row0_valid ? __ldg(q0 + ks * 8 + tq) : 0u;
+          qa[ks][1] = row1_valid ? __ldg(q1 + ks * 8 + tq) : 0u;
+          qa[ks][2] = row0_valid ? __ldg(q0 + ks * 8 + 4 + tq) : 0u;
+          qa[ks][3] = row1_valid ? __ldg(q1 + ks * 8 + 4 + tq) : 0u;
+        }
       }
-      float m[G], l[G], acc[G][DL];
+      float o[NT][4];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        m[h] = neg_inf;
-        l[h] = 0.f;
-#pragma unroll
-        for (int d = 0; d < DL; ++d) acc[h][d] = 0.f;
-      }
-      float* my_score = score + warp * 8 * G;
+      for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      float m_ref[2] = {neg_inf, neg_inf};   // per-warp exponent reference, rows g and g + 8
+      float m_true[2] = {neg_inf, neg_inf};  // unit's running max of kept tiles (tile skip)
+      float l_part[2] = {0.f, 0.f};          // this lane's share of the row sums
 
       for (int t0 = t_begin; t0 < t_end; t0 += kDecTile) {
         if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) {
@@ -224,175 +250,209 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int2 inf = info[slot];
         const int ntok = inf.x;
         const uint32_t bad = uint32_t(inf.y);
-        const __nv_bfloat16* Ks = reinterpret_cast<const __nv_bfloat16*>(smem + slot * L::kStageBytes);
-        const __nv_bfloat16* Vs = Ks + kDecTile * D;
+        const uint32_t kaddr = ring_addr + slot * L::kStageBytes;
+        const uint32_t vaddr = kaddr + L::kTileBytes;
+        const int tok_base = warp * 16;
 
-        // ---- scores of this warp's 8 tokens, reduce-scattered over the lanes
+        // ---- S = q K^T for this warp's 16 tokens (two 8-token column tiles)
+        float s[2][4];
 #pragma unroll
-        for (int bch = 0; bch < NB; ++bch) {
-          float val[V];
+        for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+        {
+          const int mi = lane >> 3, r = lane & 7;
+          const int tok = tok_base + (mi >> 1) * 8 + r;
 #pragma unroll
-          for (int tk = 0; tk < TBc; ++tk) {
-            float kx[DL];
-            load_row_slice<D>(Ks + (warp * 8 + bch * TBc + tk) * D, lane, kx);
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              float s = 0.f;
-#pragma unroll
-              for (int d = 0; d < DL; ++d) s = fmaf(qf[h][d], kx[d], s);
-              val[tk * G + h] = s;
-            }
-          }
-          int cur = V;
-#pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) {
-            if (cur > 1) {
-              const int half = cur >> 1;
-              const bool upper = (lane & off) != 0;
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                if (i < half) {
-                  const float send = upper ? val[i] : val[i + half];
-                  const float keep = upper ? val[i + half] : val[i];
-                  val[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                }
-              }
-              cur = half;
-            } else {
-              val[0] += __shfl_xor_sync(0xffffffffu, val[0], off);
-            }
-          }
-          // lane owns value index v = lane / DUP of this batch
-          if ((lane % DUP) == 0) {
-            const int v = lane / DUP;
-            const int tk = v / G;
-            const int tok = warp * 8 + bch * TBc + tk;
-            const bool vis = tok < ntok && !((bad >> (tok / p.chunk)) & 1u);
-            my_score[(bch * TBc) * G + v] = vis ? val[0] : neg_inf;
+          for (int ks = 0; ks < KS; ++ks) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kaddr + swz_off(tok, ks * 2 + (mi & 1)), b0, b1, b2, b3);
+            mma_bf16_16816(s[0], qa[ks], b0, b1);
+            mma_bf16_16816(s[1], qa[ks], b2, b3);
           }
         }
-        __syncwarp();
-        // ---- per-head max over this warp's tokens, then over the warps
-        if (lane < G) {
-          float mx = neg_inf;
+        // ---- scale to log2 units and mask tokens past the end or in invalid pages
+        const bool tile_clean = (ntok == kDecTile) && (bad == 0);
 #pragma unroll
-          for (int tk = 0; tk < 8; ++tk) mx = fmaxf(mx, my_score[tk * G + lane]);
-          red[(red_par * kDecConsumerWarps + warp) * G + lane] = mx;
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tok = tok_base + j * 8 + 2 * tq + (e & 1);
+            float v = s[j][e] * p.scale_log2;
+            if (!tile_clean && (tok >= ntok || ((bad >> (tok / p.chunk)) & 1u))) v = neg_inf;
+            s[j][e] = v;
+          }
         }
-        named_bar_sync(1, kDecConsumerWarps * 32);
-        float rmax_l = neg_inf;
-        if (lane < G) {
+        // warp-local tile row maxima (rows g, g + 8)
+        float mx[2];
+        mx[0] = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        mx[1] = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
 #pragma unroll
-          for (int w = 0; w < kDecConsumerWarps; ++w)
-            rmax_l = fmaxf(rmax_l, red[(red_par * kDecConsumerWarps + w) * G + lane]);
+        for (int r = 0; r < 2; ++r) {
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
         }
-        red_par ^= 1;
-        float r[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) r[h] = __shfl_sync(0xffffffffu, rmax_l, h);
 
         bool skip = false;
         if constexpr (SKIP) {
-          bool all_ok = true;
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const bool row_ok = (r[h] == neg_inf) || (m[h] != neg_inf && (r[h] - m[h]) < p.log2_lambda);
-            all_ok = all_ok && row_ok;
+          // tile row maxima over all four warps, then the unit-wide decision
+          if (tq == 0) {
+            red[(red_par * kDecConsumerWarps + warp) * 16 + g] = mx[0];
+            red[(red_par * kDecConsumerWarps + warp) * 16 + g + 8] = mx[1];
           }
-          skip = all_ok;
+          named_bar_sync(1, kDecConsumerWarps * 32);
+          float r[2] = {neg_inf, neg_inf};
+#pragma unroll
+          for (int w = 0; w < kDecConsumerWarps; ++w) {
+            r[0] = fmaxf(r[0], red[(red_par * kDecConsumerWarps + w) * 16 + g]);
+            r[1] = fmaxf(r[1], red[(red_par * kDecConsumerWarps + w) * 16 + g + 8]);
+          }
+          red_par ^= 1;
+          bool row_ok = true;
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const bool valid_row = rr == 0 ? row0_valid : row1_valid;
+            const bool ok_r = !valid_row || r[rr] == neg_inf ||
+                              (m_true[rr] != neg_inf && (r[rr] - m_true[rr]) < p.log2_lambda);
+            row_ok = row_ok && ok_r;
+          }
+          skip = __all_sync(0xffffffffu, row_ok) != 0;
+          if (!skip) {
+            m_true[0] = fmaxf(m_true[0], r[0]);
+            m_true[1] = fmaxf(m_true[1], r[1]);
+          }
           if (p.skip_mask && warp == 0 && lane == 0)
             p.skip_mask[(size_t(seq) * p.Hkv + kvh) * p.max_tiles + t0 / kDecTile] = skip ? 1 : 0;
         }
+
         if (!skip) {
-          float mnew[G], alpha[G];
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            mnew[h] = fmaxf(m[h], r[h]);
-            alpha[h] = (m[h] == neg_inf) ? 0.f : fast_exp2(m[h] - mnew[h]);
-          }
-          // probabilities of the owned scores, in place
-          if ((lane % DUP) == 0) {
-#pragma unroll
-            for (int bch = 0; bch < NB; ++bch) {
-              const int v = lane / DUP;
-              const int h = v % G;
-              float* sp = &my_score[(bch * TBc) * G + v];
-              const float s = *sp;
-              float mh = mnew[0];
-#pragma unroll
-              for (int hh = 1; hh < G; ++hh)
-                if (h == hh) mh = mnew[hh];
-              *sp = (s == neg_inf || mh == neg_inf) ? 0.f : fast_exp2(s - mh);
-            }
-          }
-          __syncwarp();
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            l[h] *= alpha[h];
-#pragma unroll
-            for (int d = 0; d < DL; ++d) acc[h][d] *= alpha[h];
-            m[h] = mnew[h];
-          }
-          // ---- P.V over this warp's tokens
-#pragma unroll
-          for (int tk = 0; tk < 8; ++tk) {
-            const int tok = warp * 8 + tk;
-            const bool vis = tok < ntok && !((bad >> (tok / p.chunk)) & 1u);
-            if (vis) {
-              float vx[DL];
-              load_row_slice<D>(Vs + tok * D, lane, vx);
-#pragma unroll
-              for (int h = 0; h < G; ++h) {
-                const float pr = my_score[tk * G + h];
-                l[h] += pr;
-#pragma unroll
-                for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(pr, vx[d], acc[h][d]);
+          // zero the V rows of masked tokens so that 0 * (stale or NaN) cannot reach O
+          if (!tile_clean) {
+            bool any_masked = false;
+            for (int t = 0; t < 16; ++t) {
+              const int tok = tok_base + t;
+              const bool masked = tok >= ntok || ((bad >> (tok / p.chunk)) & 1u);
+              any_masked |= masked;
+              if (masked) {
+                for (int c = lane; c < D / 8; c += 32)
+                  *reinterpret_cast<uint4*>(smem + slot * L::kStageBytes + L::kTileBytes + swz_off(tok, c)) =
+                      make_uint4(0, 0, 0, 0);
               }
             }
+            if (any_masked) __syncwarp();
           }
+          // reference maximum: raised only when the tile exceeds it by more than 2^8
+          float alpha[2] = {1.f, 1.f};
+          bool raised = false;
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            if (mx[r] != neg_inf && (m_ref[r] == neg_inf || mx[r] > m_ref[r] + kDecRescaleThreshold)) {
+              alpha[r] = (m_ref[r] == neg_inf) ? 0.f : fast_exp2(m_ref[r] - mx[r]);
+              m_ref[r] = mx[r];
+              raised = true;
+            }
+          }
+          if (__any_sync(0xffffffffu, raised)) {
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
+              o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
+            }
+            l_part[0] *= alpha[0];
+            l_part[1] *= alpha[1];
+          }
+          // probabilities, packed as the A operand of P V
+          uint32_t pa[4];
+          {
+            const float off0 = m_ref[0] == neg_inf ? 0.f : m_ref[0];
+            const float off1 = m_ref[1] == neg_inf ? 0.f : m_ref[1];
+            float pr[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              pr[j][0] = row0_valid ? fast_exp2(s[j][0] - off0) : 0.f;
+              pr[j][1] = row0_valid ? fast_exp2(s[j][1] - off0) : 0.f;
+              pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
+              pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
+            }
+            l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+            l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+            pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+            pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+            pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+            pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+          }
+          // ---- O += P V over this warp's 16 tokens
+          {
+            const int mi = lane >> 3, r = lane & 7;
+            const int tok = tok_base + (mi & 1) * 8 + r;
+#pragma unroll
+            for (int n2 = 0; n2 < NT / 2; ++n2) {
+              uint32_t v0, v1, v2, v3;
+              ldsm_x4_t(vaddr + swz_off(tok, n2 * 2 + (mi >> 1)), v0, v1, v2, v3);
+              mma_bf16_16816(o[2 * n2], pa, v0, v1);
+              mma_bf16_16816(o[2 * n2 + 1], pa, v2, v3);
+            }
+          }
+          if (!tile_clean) fence_proxy_async_smem();  // zeroed rows before the next TMA write
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
-        if (++slot == kDecStages) { slot = 0; phase ^= 1u; }
+        if (++slot == NS) { slot = 0; phase ^= 1u; }
       }
       if (!ok) break;
 
-      // ---- combine the eight warps' (l, O) for this item and write the split result
+      // ---- merge the four warps' (m, l, O) in a fixed order and write the split result
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+      for (int r = 0; r < 2; ++r) {
+        l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 1);
+        l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 2);
+      }
+      if (row0_valid) {
 #pragma unroll
-        for (int d = 0; d < DL; ++d) atomicAdd(&comb_o[h * D + lane * DL + d], acc[h][d]);
-        if (lane == 0) atomicAdd(&comb_l[item_par * G + h], l[h]);
+        for (int n = 0; n < NT; ++n) {
+          float* dst = comb_o + (warp * G + g) * D + n * 8 + 2 * tq;
+          dst[0] = o[n][0];
+          dst[1] = o[n][1];
+        }
+        if (tq == 0) { comb_m[warp * G + g] = m_ref[0]; comb_l[warp * G + g] = l_part[0]; }
+      }
+      if (row1_valid) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          float* dst = comb_o + (warp * G + g + 8) * D + n * 8 + 2 * tq;
+          dst[0] = o[n][2];
+          dst[1] = o[n][3];
+        }
+        if (tq == 0) { comb_m[warp * G + g + 8] = m_ref[1]; comb_l[warp * G + g + 8] = l_part[1]; }
       }
       named_bar_sync(1, kDecConsumerWarps * 32);
       const int tid = threadIdx.x;
       for (int i = tid; i < G * D; i += kDecConsumerWarps * 32) {
         const int h = i / D, d = i % D;
-        const float lsum = comb_l[item_par * G + h];
-        const float val = lsum > 0.f ? comb_o[i] / lsum : 0.f;  // 0 only if every page was invalid
-        comb_o[i] = 0.f;
+        float M = neg_inf;
+#pragma unroll
+        for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, comb_m[w * G + h]);
+        float lsum = 0.f, osum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecConsumerWarps; ++w) {
+          const float mw = comb_m[w * G + h];
+          const float e = (mw == neg_inf) ? 0.f : fast_exp2(mw - M);
+          lsum += e * comb_l[w * G + h];
+          osum += e * comb_o[(w * G + h) * D + d];
+        }
+        const float val = lsum > 0.f ? osum / lsum : 0.f;  // 0 only if every page was invalid
         const int hq = kvh * G + h;
         if (n_splits == 1)
           p.o[(size_t(seq) * p.Hq + hq) * D + d] = __float2bfloat16_rn(val);
         else
           p.ws_o[((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + d] = val;
-      }
-      if (tid < G) {
-        const float lsum = comb_l[item_par * G + tid];
-        float mh = m[0];
-#pragma unroll
-        for (int hh = 1; hh < G; ++hh)
-          if (tid == hh) mh = m[hh];
-        const float lse2 = lsum > 0.f ? mh + __log2f(lsum) : -__int_as_float(0x7f800000);
-        const int hq = kvh * G + tid;
-        if (n_splits == 1) {
-          if (p.lse) p.lse[size_t(seq) * p.Hq + hq] = lse2 * 0.69314718055994531f;
-        } else {
-          p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lse2;
+        if (d == 0) {
+          const float lse2 = lsum > 0.f ? M + __log2f(lsum) : neg_inf;
+          if (n_splits == 1) {
+            if (p.lse) p.lse[size_t(seq) * p.Hq + hq] = lse2 * 0.69314718055994531f;
+          } else {
+            p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lse2;
+          }
         }
-        comb_l[(item_par ^ 1) * G + tid] = 0.f;
       }
-      item_par ^= 1;
     }
   }
   __syncwarp();
@@ -430,16 +490,18 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeParams p)
   for (int d = 0; d < DL; ++d) acc[d] = 0.f;
   float wsum = 0.f;
   for (int s = 0; s < n_splits; ++s) {
-    const float w = fast_exp2(lse_base[size_t(s) * p.Hq] - mx);
+    const float ls = lse_base[size_t(s) * p.Hq];
+    const float w = (ls == neg_inf) ? 0.f : fast_exp2(ls - mx);
     const float* orow_s = p.ws_o + ((size_t(seq) * p.max_splits + s) * p.Hq + hq) * D + lane * DL;
     wsum += w;
 #pragma unroll
     for (int d = 0; d < DL; ++d) acc[d] = fmaf(w, orow_s[d], acc[d]);
   }
-  const float inv = 1.f / wsum;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
 #pragma unroll
   for (int d = 0; d < DL; ++d) orow[lane * DL + d] = __float2bfloat16_rn(acc[d] * inv);
-  if (p.lse && lane == 0) p.lse[size_t(seq) * p.Hq + hq] = (mx + __log2f(wsum)) * 0.69314718055994531f;
+  if (p.lse && lane == 0)
+    p.lse[size_t(seq) * p.Hq + hq] = wsum > 0.f ? (mx + __log2f(wsum)) * 0.69314718055994531f : neg_inf;
 }
 
 }  // namespace attn
