@@ -93,6 +93,11 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
                    int sms, cudaStream_t stream) {
   auto kernel = prefill_kernel<D, CAUSAL, SKIP>;
   constexpr int smem = PrefillSmem<D>::kDynamic;
+  // The kernel moves registers between warpgroups with setmaxnreg; the block's
+  // launch allocation must cover the split or the increase would never return.
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (attr.numRegs * kPfThreads < kPfRegPoolNeeded) return ATTN_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const long long grid = p.num_items < sms ? p.num_items : sms;
