@@ -48,8 +48,12 @@ SIGNATURES = {
     "attn_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                _P, _SZ, _P, _P, _P]),
+    "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
+                                       _P, _P, _P]),
     "attn_read_device_status": (_I, [ctypes.POINTER(_I), _I]),
 }
+
+NOALLOC_SCRATCH_BYTES = 16 << 20   # ATTN_NOALLOC_SCRATCH_BYTES
 
 
 def lib_path() -> str:
@@ -215,3 +219,29 @@ def decode_paged_blasst(q, k_pages, v_pages, block_table, seq_lens, lam: float, 
     """Paged decode with the BLASST tile skip. Returns (o, lse, skip_mask)."""
     return _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens, out, lse,
                    workspace, skip_mask, device_status, return_lse, stream)
+
+
+def decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale=None, split_tokens: int = 1024,
+                         out=None, lse=None, device_status=None, return_lse=True, stream=None):
+    """Dense paged decode through the entry point that allocates nothing: the
+    split partials go to the library's fixed 16 MiB device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory at decode
+    time). Calls on one device share that scratch, so they must not overlap on
+    the GPU. Returns (o, lse)."""
+    _need(q, torch.bfloat16, 3, "q")
+    _need(k_pages, torch.bfloat16, 4, "k_pages")
+    _need(v_pages, torch.bfloat16, 4, "v_pages")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    N, Hq, D = q.shape
+    P, page_size, Hkv, _ = k_pages.shape
+    scale = default_scale(D) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    if lse is None and return_lse:
+        lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_decode_paged_noalloc(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), N, Hq, Hkv, D, page_size,
+        block_table.shape[1], P, scale, 0.0, split_tokens, _ptr(o), _ptr(lse), None, _ptr(device_status),
+        _stream_handle(stream))
+    _check(st, "attn_decode_paged_noalloc")
+    return o, lse

@@ -291,6 +291,49 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
                   : dispatch_decode_g<64, false>(G, tk, tv, p, sms, s);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ decode without a workspace
+
+// The fixed scratch of attn_decode_paged_noalloc (see the header): every device
+// that loads the library holds it; each call's split partials are written
+// before they are read, so it never needs clearing.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per device.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_noalloc_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return ATTN_ERR_CUDA;
+    g_noalloc_scratch_addr[dev] = ptr;
+  }
+  *out = g_noalloc_scratch_addr[dev];
+  return ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                              const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
+                              int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens,
+                              void* o, float* lse, uint8_t* skip_mask, int* device_status, void* stream) {
+  const size_t need = attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens);
+  if (need == 0 || need > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (int st = noalloc_scratch(&scratch)) return st;
+  return attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_seqs, Hq, Hkv, D, page_size,
+                           max_pages_per_seq, num_pages, scale, lambda, split_tokens, o, lse, scratch,
+                           ATTN_NOALLOC_SCRATCH_BYTES, skip_mask, device_status, stream);
+}
+
 int attn_read_device_status(int* status_out, int clear) {
   if (!status_out) return ATTN_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;

@@ -152,6 +152,41 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                       uint8_t* skip_mask, int* device_status, void* stream);
 
 /*
+ * attn_decode_paged_noalloc -- attn_decode_paged without a caller-provided
+ * workspace. (Library plumbing: the pages describe no counterpart.)
+ *
+ * Some callers cannot allocate device memory when they decode: a serving loop
+ * that reserves all of the device memory for its KV-cache pool at start-up,
+ * or a latency-critical thread that must not call cudaMalloc (which may
+ * synchronise the device). This entry point allocates nothing. Its split
+ * partials live in a fixed array of ATTN_NOALLOC_SCRATCH_BYTES (16 MiB) of
+ * device memory inside the library, which every device that loads the library
+ * holds until the process exits.
+ *
+ * Arguments, layouts, results and errors are those of attn_decode_paged,
+ * minus workspace / workspace_bytes. A call whose
+ * attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size,
+ * split_tokens) exceeds ATTN_NOALLOC_SCRATCH_BYTES returns
+ * ATTN_ERR_INVALID_ARG before anything is enqueued (use a larger split_tokens
+ * or attn_decode_paged).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. Every call on a device shares the one array and leaves its
+ * contents behind (nothing in it needs clearing between calls), so calls that
+ * may run at the same time on the GPU -- on different streams without an
+ * ordering between them -- race on it: order them, or use attn_decode_paged
+ * with separate workspaces.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                              const int32_t* block_table, const int32_t* seq_lens,
+                              int num_seqs, int Hq, int Hkv, int D, int page_size,
+                              int max_pages_per_seq, int num_pages, float scale, float lambda,
+                              int split_tokens, void* o, float* lse,
+                              uint8_t* skip_mask, int* device_status, void* stream);
+
+/*
  * attn_read_device_status -- read (and, if clear != 0, reset to ATTN_OK) the
  * library's device status word on the current device. Synchronises the
  * device. Every kernel of the library ORs a device-side error into it.
