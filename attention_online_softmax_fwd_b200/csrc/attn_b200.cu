@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_heads.cuh"
 #include "prefill.cuh"
 
 using namespace attn;
@@ -72,6 +73,21 @@ int encode_map(CUtensorMap* map, const void* base, const uint64_t dims[4], const
   cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d, s, b, elem_strides,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
+}
+
+// 5-D bf16 tensor map with the 128-byte swizzle. dims/box innermost first; strides in bytes for dims 1..4.
+int encode_map5(CUtensorMap* map, const void* base, const uint64_t dims[5], const uint64_t strides[4],
+                const uint32_t box[5]) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return ATTN_ERR_CUDA;
+  const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  cuuint64_t d[5] = {dims[0], dims[1], dims[2], dims[3], dims[4]};
+  cuuint64_t s[4] = {strides[0], strides[1], strides[2], strides[3]};
+  cuuint32_t b[5] = {box[0], box[1], box[2], box[3], box[4]};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), d, s, b, elem_strides,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
 }
@@ -153,6 +169,9 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
 
 // ------------------------------------------------------------------ decode
 
+// decode workspace: [work-ticket counter, 256 B][partial O][partial log2-sum-exp]
+constexpr size_t kWsHeader = 256;
+
 bool valid_page_size(int ps) { return ps == 16 || ps == 32 || ps == 64 || ps == 128 || ps == 256; }
 
 long long max_splits_of(int max_pages, int page_size, int split_tokens) {
@@ -187,6 +206,42 @@ int dispatch_decode_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const
     case 16: return launch_decode<D, 16, SKIP>(tk, tv, p, sms, s);
     default: return ATTN_ERR_UNSUPPORTED;
   }
+}
+
+template <int D, int G, int HG>
+int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int* ticket_counter,
+                        int sms, cudaStream_t stream) {
+  auto kernel = decode_heads_kernel<D, G, HG>;
+  constexpr int smem = DecodeHeadsSmem<D, G, HG>::kDynamic;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
+  const long long grid = items < sms ? items : sms;
+  kernel<<<dim3(unsigned(grid)), dim3((HG + 1) * 32), smem, stream>>>(tk, tv, p, ticket_counter);
+  if (int st = launch_status()) return st;
+  const long long pairs = (long long)p.num_seqs * p.Hq;
+  decode_merge_kernel<D><<<dim3(unsigned((pairs + 7) / 8)), dim3(256), 0, stream>>>(p);
+  return launch_status();
+}
+
+template <int D, int HG>
+int dispatch_decode_heads_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int* ctr,
+                            int sms, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_decode_heads<D, 1, HG>(tk, tv, p, ctr, sms, s);
+    case 2: return launch_decode_heads<D, 2, HG>(tk, tv, p, ctr, sms, s);
+    case 4: return launch_decode_heads<D, 4, HG>(tk, tv, p, ctr, sms, s);
+    case 8: return launch_decode_heads<D, 8, HG>(tk, tv, p, ctr, sms, s);
+    case 16: return launch_decode_heads<D, 16, HG>(tk, tv, p, ctr, sms, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+template <int D>
+int dispatch_decode_heads(int G, int hg, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                          int* ctr, int sms, cudaStream_t s) {
+  return hg == 8 ? dispatch_decode_heads_g<D, 8>(G, tk, tv, p, ctr, sms, s)
+                 : dispatch_decode_heads_g<D, 4>(G, tk, tv, p, ctr, sms, s);
 }
 
 }  // namespace
@@ -227,7 +282,7 @@ size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_pe
   const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
   const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
   const size_t o_bytes_aligned = (o_bytes + 255) / 256 * 256;
-  return o_bytes_aligned + size_t(num_seqs) * ms * Hq * sizeof(float);
+  return kWsHeader + o_bytes_aligned + size_t(num_seqs) * ms * Hq * sizeof(float);
 }
 
 int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
@@ -259,9 +314,10 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
-  p.ws_o = static_cast<float*>(workspace);
+  int* ticket_counter = static_cast<int*>(workspace);
+  p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader);
   const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
-  p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (o_bytes + 255) / 256 * 256);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader + (o_bytes + 255) / 256 * 256);
   p.skip_mask = skip_mask;
   p.status = device_status;
   p.num_seqs = num_seqs; p.Hq = Hq; p.Hkv = Hkv;
@@ -274,16 +330,29 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   p.log2_lambda = lambda > 0.f ? std::log2(lambda) : -INFINITY;
   p.num_items = (long long)num_seqs * ms * Hkv;
 
-  // page pool [P][page_size][Hkv][D] as a 4-D map {D, Hkv, page_size, P}; box = 64 columns of one head
-  // for `chunk` tokens, written with the 128-byte swizzle
-  const uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(page_size), uint64_t(num_pages)};
-  const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(Hkv) * D * 2, uint64_t(page_size) * Hkv * D * 2};
-  const uint32_t box[4] = {64, 1, uint32_t(p.chunk), 1};
+  // page pool [P][page_size][Hkv][D] as a 5-D map {64, D/64, Hkv, page_size, P}; box = the whole head
+  // dimension of one head for `chunk` tokens, written as 128-byte rows with the 128-byte swizzle
+  const uint64_t dims[5] = {64, uint64_t(D / 64), uint64_t(Hkv), uint64_t(page_size), uint64_t(num_pages)};
+  const uint64_t strides[4] = {128, uint64_t(D) * 2, uint64_t(Hkv) * D * 2, uint64_t(page_size) * Hkv * D * 2};
+  const uint32_t box[5] = {64, uint32_t(D / 64), 1, uint32_t(p.chunk), 1};
   CUtensorMap tk, tv;
-  if (int st = encode_map(&tk, k_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return st;
-  if (int st = encode_map(&tv, v_pages, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return st;
+  if (int st = encode_map5(&tk, k_pages, dims, strides, box)) return st;
+  if (int st = encode_map5(&tv, v_pages, dims, strides, box)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool use_skip = lambda > 0.f || skip_mask != nullptr;
+  const int hg = Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0);
+  if (!use_skip && hg > 0) {
+    // dense: one item per group of hg KV heads, 16-token stages covering all of them
+    const uint64_t hdims[5] = {64, uint64_t(D / 64), uint64_t(page_size), uint64_t(Hkv), uint64_t(num_pages)};
+    const uint64_t hstrides[4] = {128, uint64_t(Hkv) * D * 2, uint64_t(D) * 2, uint64_t(page_size) * Hkv * D * 2};
+    const uint32_t hbox[5] = {64, uint32_t(D / 64), uint32_t(kDhChunk), uint32_t(hg), 1};
+    CUtensorMap hk, hv;
+    if (int st = encode_map5(&hk, k_pages, hdims, hstrides, hbox)) return st;
+    if (int st = encode_map5(&hv, v_pages, hdims, hstrides, hbox)) return st;
+    if (cudaMemsetAsync(ticket_counter, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (D == 128) return dispatch_decode_heads<128>(G, hg, hk, hv, p, ticket_counter, sms, s);
+    return dispatch_decode_heads<64>(G, hg, hk, hv, p, ticket_counter, sms, s);
+  }
   if (D == 128)
     return use_skip ? dispatch_decode_g<128, true>(G, tk, tv, p, sms, s)
                     : dispatch_decode_g<128, false>(G, tk, tv, p, sms, s);

@@ -3,9 +3,14 @@
 // Work item = (sequence, split, KV head). A persistent CTA walks its items in
 // a strided order. One producer warp streams the item's 64-token tiles of K
 // and V from the page pool into a shared-memory ring with TMA, one copy per
-// (page chunk, 64-column half, K|V), addressed through the block table. The
-// copies use the 128-byte swizzle so that the consumers' ldmatrix reads are
-// free of bank conflicts.
+// (page chunk, K|V), addressed through the block table. The page pool is seen
+// as 5-D {64 columns, D/64 column blocks, head, slot, page} so that one copy
+// moves a chunk's whole head dimension; it lands as rows of 128 bytes
+// (token-major, column block minor) with the 128-byte swizzle, which keeps the
+// consumers' ldmatrix reads to at most two-way bank conflicts. The producer reads the next item's length and first
+// block-table window while it streams the current item, and ships each item's
+// query rows (one bulk copy) and metadata with its first tile, so neither side
+// waits on a dependent global load when an item starts.
 //
 // Four consumer warps each take 16 tokens of a tile. The G query heads that
 // share the KV head are the rows of a 16-row operand (rows >= G are zero), so
@@ -48,22 +53,38 @@ constexpr int kDecConsumerWarps = 4;  // 16 tokens of each tile per warp
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
 constexpr float kDecRescaleThreshold = 8.0f;  // log2 units
 
+// What the producer tells the consumers about a stage.
+struct TileInfo {
+  int seq, split, kvh, t0;
+  int ntok;   // valid tokens of the tile from t0
+  int bad;    // bit c: page chunk c was outside the pool (not loaded)
+  int flags;  // bit 0: first tile of the item (its query rows are in the stage), bit 1: last tile,
+              // bit 2: no tile, this CTA's work is done
+  int len;    // sequence length (clamped to the block table's capacity)
+};
+
 template <int D, int G>
 struct DecodeSmem {
-  static constexpr int kHalfBytes = kDecTile * 128;            // 64 tokens x 64 columns, 128B-swizzled
   static constexpr int kTileBytes = kDecTile * D * 2;          // one K or V tile
-  static constexpr int kStageBytes = 2 * kTileBytes;           // K then V
-  static constexpr int kStages = D == 128 ? 6 : 12;
+  static constexpr int kQBytes = G * D * 2;                    // the item's query rows
+  static constexpr int kStageBytes = (2 * kTileBytes + kQBytes + 1023) / 1024 * 1024;  // K, V, q
+  // as many stages (at most 6 for D = 128, 11 for D = 64) as fit beside the combine buffers
+  static constexpr int kFixed = 16 * 12 + 4 * 2 * kDecConsumerWarps * 16 + 8 * kDecConsumerWarps * G +
+                                4 * kDecConsumerWarps * G * D + 1024 + 64;
+  static constexpr int kFit = (232448 - kFixed) / (kStageBytes + 48);
+  static constexpr int kStages = (D == 128 ? 6 : 11) < kFit ? (D == 128 ? 6 : 11) : kFit;
   static constexpr int kRing = kStages * kStageBytes;
   static constexpr int kFull = kRing;                                   // mbarriers
   static constexpr int kEmpty = kFull + 8 * kStages;
-  static constexpr int kInfo = kEmpty + 8 * kStages;                    // int2 per stage
-  static constexpr int kRed = kInfo + 8 * kStages;                      // [2][warps][16] floats
+  static constexpr int kInfo = kEmpty + 8 * kStages;                    // TileInfo per stage
+  static constexpr int kRed = kInfo + 32 * kStages;                     // [2][warps][16] floats
   static constexpr int kCombM = kRed + 4 * 2 * kDecConsumerWarps * 16;  // [warps][G] floats
   static constexpr int kCombL = kCombM + 4 * kDecConsumerWarps * G;     // [warps][G] floats
   static constexpr int kCombO = (kCombL + 4 * kDecConsumerWarps * G + 15) / 16 * 16;  // [warps][G][D]
   static constexpr int kTotal = kCombO + 4 * kDecConsumerWarps * G * D;
   static constexpr int kDynamic = kTotal + 1024;                        // slack for alignment
+  static_assert(kDynamic <= 232448, "shared memory per block");
+  static_assert(kStages >= 2, "ring depth");
 };
 
 __device__ __forceinline__ void decode_item_coords(long long item, int Hkv, int max_splits, int& seq, int& split,
@@ -74,9 +95,12 @@ __device__ __forceinline__ void decode_item_coords(long long item, int Hkv, int 
   seq = int(rest / max_splits);
 }
 
-// Byte offset of 16-byte chunk `c` (0 .. D/8-1) of token row `r` in a swizzled tile.
+// Byte offset of 16-byte chunk `c` (0 .. D/8-1) of token `r` in a swizzled K or V
+// tile: 128-byte row (r * D/64 + c / 8), unit (c mod 8) XOR (row mod 8).
+template <int D>
 __device__ __forceinline__ uint32_t swz_off(int r, int c) {
-  return uint32_t((c >> 3) * (kDecTile * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+  const int row = r * (D / 64) + (c >> 3);
+  return uint32_t(row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
 
 template <int D, int G, bool SKIP>
@@ -93,7 +117,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kFull);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::kEmpty);
-  int2* info = reinterpret_cast<int2*>(smem + L::kInfo);
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + L::kInfo);
   float* red = reinterpret_cast<float*>(smem + L::kRed);
   float* comb_m = reinterpret_cast<float*>(smem + L::kCombM);
   float* comb_l = reinterpret_cast<float*>(smem + L::kCombL);
@@ -127,10 +151,35 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     uint32_t pending = 0;  // stages with copies issued, for the abort path
     uint32_t pending_phase = 0;
     bool ok = true;
+    // The next candidate item's length and first block-table window are loaded
+    // one item ahead; the window does not depend on the length (entries past
+    // the sequence end are read but never used).
+    int nx_len = 0, nx_win = -1;
+    {
+      const long long it = blockIdx.x;
+      if (it < p.num_items) {
+        int sq, sp, kh;
+        decode_item_coords(it, p.Hkv, p.max_splits, sq, sp, kh);
+        nx_len = __ldg(&p.seq_lens[sq]);
+        const int e = (((sp * p.split_tokens) / p.page_size) & ~31) + lane;
+        nx_win = e < p.max_pages ? __ldg(&p.block_table[size_t(sq) * p.max_pages + e]) : -1;
+      }
+    }
     for (long long item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
       int seq, split, kvh;
       decode_item_coords(item, p.Hkv, p.max_splits, seq, split, kvh);
-      int len = __ldg(&p.seq_lens[seq]);
+      int len = nx_len;
+      int win_cur = nx_win;
+      {
+        const long long it = item + gridDim.x;
+        if (it < p.num_items) {
+          int sq, sp, kh;
+          decode_item_coords(it, p.Hkv, p.max_splits, sq, sp, kh);
+          nx_len = __ldg(&p.seq_lens[sq]);
+          const int e = (((sp * p.split_tokens) / p.page_size) & ~31) + lane;
+          nx_win = e < p.max_pages ? __ldg(&p.block_table[size_t(sq) * p.max_pages + e]) : -1;
+        }
+      }
       if (len > capacity || len < 0) {
         if (lane == 0 && split == 0 && kvh == 0) raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
         len = len < 0 ? 0 : capacity;
@@ -139,22 +188,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (t_begin >= len) continue;
       const int t_end = min(t_begin + p.split_tokens, len);
       const int32_t* bt_row = p.block_table + size_t(seq) * p.max_pages;
-      // Block-table entries are fetched 32 at a time (one per lane), one window
-      // ahead, so that a tile's page ids are a shuffle away when it is issued.
-      const int n_entries = (len + p.page_size - 1) / p.page_size;
-      auto load_window = [&](int w) {
-        const int e = w * 32 + lane;
-        return e < n_entries ? __ldg(&bt_row[e]) : -1;
-      };
       int win = (t_begin / p.page_size) >> 5;
-      int win_cur = load_window(win);
-      int win_next = load_window(win + 1);
+      int win_next;
+      {
+        const int e = (win + 1) * 32 + lane;
+        win_next = e < p.max_pages ? __ldg(&bt_row[e]) : -1;
+      }
+      const __nv_bfloat16* qsrc = p.q + (size_t(seq) * p.Hq + size_t(kvh) * G) * D;
       for (int t0 = t_begin; t0 < t_end; t0 += kDecTile) {
         const int e0 = t0 / p.page_size;  // first entry of this tile; a tile never straddles a window
         if ((e0 >> 5) != win) {
           win = e0 >> 5;
           win_cur = win_next;
-          win_next = load_window(win + 1);
+          const int e = (win + 1) * 32 + lane;
+          win_next = e < p.max_pages ? __ldg(&bt_row[e]) : -1;
         }
         if (!mbar_wait(&empty[slot], phase ^ 1u, &abort_flag, p.status)) { ok = false; break; }
         const int p0 = t0 + lane * p.chunk;
@@ -170,26 +217,44 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         const uint32_t valid_mask = __ballot_sync(0xffffffffu, valid);
         const uint32_t bad_mask = __ballot_sync(0xffffffffu, bad);
+        const bool first = t0 == t_begin;
+        uint8_t* stage = smem + slot * L::kStageBytes;
         if (lane == 0) {
           if (bad_mask) raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
-          info[slot] = make_int2(min(kDecTile, len - t0), int(bad_mask));
-          mbar_arrive_expect_tx(&full[slot], __popc(valid_mask) * chunk_bytes * 2);
+          TileInfo ti;
+          ti.seq = seq; ti.split = split; ti.kvh = kvh; ti.t0 = t0;
+          ti.ntok = min(kDecTile, len - t0);
+          ti.bad = int(bad_mask);
+          ti.flags = (first ? 1 : 0) | (t0 + kDecTile >= t_end ? 2 : 0);
+          ti.len = len;
+          info[slot] = ti;
+          mbar_arrive_expect_tx(&full[slot], __popc(valid_mask) * chunk_bytes * 2 + (first ? uint32_t(L::kQBytes) : 0u));
+          if (first) bulk_load(stage + 2 * L::kTileBytes, qsrc, uint32_t(L::kQBytes), &full[slot]);
         }
         __syncwarp();
         if (valid) {
-          uint8_t* kbase = smem + slot * L::kStageBytes;
-          uint8_t* vbase = kbase + L::kTileBytes;
-          const int row0 = lane * p.chunk;
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h) {
-            tma_load_4d(kbase + h * L::kHalfBytes + row0 * 128, &tm_k, &full[slot], h * 64, kvh, in_page, page);
-            tma_load_4d(vbase + h * L::kHalfBytes + row0 * 128, &tm_v, &full[slot], h * 64, kvh, in_page, page);
-          }
+          uint8_t* kbase = stage;
+          uint8_t* vbase = stage + L::kTileBytes;
+          const uint32_t off = uint32_t(lane) * chunk_bytes;   // the chunk's first token row
+          tma_load_5d(kbase + off, &tm_k, &full[slot], 0, 0, kvh, in_page, page);
+          tma_load_5d(vbase + off, &tm_v, &full[slot], 0, 0, kvh, in_page, page);
         }
         pending |= 1u << slot;
         pending_phase = (pending_phase & ~(1u << slot)) | (phase << slot);
         if (++slot == NS) { slot = 0; phase ^= 1u; }
       }
+    }
+    if (ok && mbar_wait(&empty[slot], phase ^ 1u, &abort_flag, p.status)) {
+      // end-of-work marker: a stage with no copies
+      if (lane == 0) {
+        TileInfo ti{};
+        ti.flags = 4;
+        info[slot] = ti;
+        mbar_arrive_expect_tx(&full[slot], 0u);
+      }
+      __syncwarp();
+    } else {
+      ok = false;
     }
     if (!ok && lane == 0) {
       for (int s = 0; s < NS; ++s)
@@ -209,195 +274,203 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     bool ok = true;
     const uint32_t ring_addr = smem_u32(smem);
 
-    for (long long item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
-      int seq, split, kvh;
-      decode_item_coords(item, p.Hkv, p.max_splits, seq, split, kvh);
-      int len = __ldg(&p.seq_lens[seq]);
-      len = len < 0 ? 0 : min(len, capacity);
-      const int t_begin = split * p.split_tokens;
-      if (t_begin >= len) continue;
-      const int t_end = min(t_begin + p.split_tokens, len);
-      const int n_splits = (len + p.split_tokens - 1) / p.split_tokens;
+    // The consumers follow the stages the producer fills, until a stage marked
+    // as the end of this CTA's work.
+    int seq = 0, split = 0, kvh = 0, n_splits = 0;
+    uint32_t qa[KS][4];
+    float o[NT][4];
+    float m_ref[2] = {neg_inf, neg_inf};   // per-warp exponent reference, rows g and g + 8
+    float m_true[2] = {neg_inf, neg_inf};  // unit's running max of kept tiles (tile skip)
+    float l_part[2] = {0.f, 0.f};          // this lane's share of the row sums
 
-      // q of the G heads as the A operand (rows >= G are zero)
-      uint32_t qa[KS][4];
-      {
+    while (ok) {
+      if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) {
+        ok = false;
+        break;
+      }
+      const TileInfo ti = info[slot];
+      if (ti.flags & 4) break;   // end of work
+      const int ntok = ti.ntok;
+      const uint32_t bad = uint32_t(ti.bad);
+      const int t0 = ti.t0;
+      if (ti.flags & 1) {
+        // first tile of an item: its query rows (A operand, rows >= G zero) came with this stage
+        seq = ti.seq; split = ti.split; kvh = ti.kvh;
+        n_splits = (ti.len + p.split_tokens - 1) / p.split_tokens;
+        const uint32_t* qs = reinterpret_cast<const uint32_t*>(smem + slot * L::kStageBytes + 2 * L::kTileBytes);
         const int h0 = row0_valid ? g : 0, h1 = row1_valid ? g + 8 : 0;
-        const uint32_t* q0 =
-            reinterpret_cast<const uint32_t*>(p.q + (size_t(seq) * p.Hq + size_t(kvh) * G + h0) * D);
-        const uint32_t* q1 =
-            reinterpret_cast<const uint32_t*>(p.q + (size_t(seq) * p.Hq + size_t(kvh) * G + h1) * D);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
-          qa[ks][0] = row0_valid ? __ldg(q0 + ks * 8 + tq) : 0u;
-          qa[ks][1] = row1_valid ? __ldg(q1 + ks * 8 + tq) : 0u;
-          qa[ks][2] = row0_valid ? __ldg(q0 + ks * 8 + 4 + tq) : 0u;
-          qa[ks][3] = row1_valid ? __ldg(q1 + ks * 8 + 4 + tq) : 0u;
+          qa[ks][0] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + tq] : 0u;
+          qa[ks][1] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + tq] : 0u;
+          qa[ks][2] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + 4 + tq] : 0u;
+          qa[ks][3] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + 4 + tq] : 0u;
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+        m_ref[0] = m_ref[1] = neg_inf;
+        m_true[0] = m_true[1] = neg_inf;
+        l_part[0] = l_part[1] = 0.f;
+      }
+      const bool last_tile = (ti.flags & 2) != 0;
+      const uint32_t kaddr = ring_addr + slot * L::kStageBytes;
+      const uint32_t vaddr = kaddr + L::kTileBytes;
+      const int tok_base = warp * 16;
+
+      // ---- S = q K^T for this warp's 16 tokens (two 8-token column tiles); the
+      // k-steps alternate between two accumulators per column tile so that
+      // consecutive MMAs do not wait on each other
+      float s[2][4];
+      {
+        float sp[2][2][4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int a = 0; a < 2; ++a) sp[j][a][0] = sp[j][a][1] = sp[j][a][2] = sp[j][a][3] = 0.f;
+        const int mi = lane >> 3, r = lane & 7;
+        const int tok = tok_base + (mi >> 1) * 8 + r;
+        uint32_t b[KS][4];
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) ldsm_x4(kaddr + swz_off<D>(tok, ks * 2 + (mi & 1)), b[ks][0], b[ks][1], b[ks][2], b[ks][3]);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          mma_bf16_16816(sp[0][ks & 1], qa[ks], b[ks][0], b[ks][1]);
+          mma_bf16_16816(sp[1][ks & 1], qa[ks], b[ks][2], b[ks][3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[j][e] = sp[j][0][e] + sp[j][1][e];
+      }
+      // ---- scale to log2 units and mask tokens past the end or in invalid pages
+      const bool tile_clean = (ntok == kDecTile) && (bad == 0);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = tok_base + j * 8 + 2 * tq + (e & 1);
+          float v = s[j][e] * p.scale_log2;
+          if (!tile_clean && (tok >= ntok || ((bad >> (tok / p.chunk)) & 1u))) v = neg_inf;
+          s[j][e] = v;
         }
       }
-      float o[NT][4];
+      // warp-local tile row maxima (rows g, g + 8)
+      float mx[2];
+      mx[0] = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+      mx[1] = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
 #pragma unroll
-      for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-      float m_ref[2] = {neg_inf, neg_inf};   // per-warp exponent reference, rows g and g + 8
-      float m_true[2] = {neg_inf, neg_inf};  // unit's running max of kept tiles (tile skip)
-      float l_part[2] = {0.f, 0.f};          // this lane's share of the row sums
+      for (int r = 0; r < 2; ++r) {
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+      }
 
-      for (int t0 = t_begin; t0 < t_end; t0 += kDecTile) {
-        if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) {
-          ok = false;
-          break;
+      bool skip = false;
+      if constexpr (SKIP) {
+        // tile row maxima over all four warps, then the unit-wide decision
+        if (tq == 0) {
+          red[(red_par * kDecConsumerWarps + warp) * 16 + g] = mx[0];
+          red[(red_par * kDecConsumerWarps + warp) * 16 + g + 8] = mx[1];
         }
-        const int2 inf = info[slot];
-        const int ntok = inf.x;
-        const uint32_t bad = uint32_t(inf.y);
-        const uint32_t kaddr = ring_addr + slot * L::kStageBytes;
-        const uint32_t vaddr = kaddr + L::kTileBytes;
-        const int tok_base = warp * 16;
+        named_bar_sync(1, kDecConsumerWarps * 32);
+        float r[2] = {neg_inf, neg_inf};
+#pragma unroll
+        for (int w = 0; w < kDecConsumerWarps; ++w) {
+          r[0] = fmaxf(r[0], red[(red_par * kDecConsumerWarps + w) * 16 + g]);
+          r[1] = fmaxf(r[1], red[(red_par * kDecConsumerWarps + w) * 16 + g + 8]);
+        }
+        red_par ^= 1;
+        bool row_ok = true;
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const bool valid_row = rr == 0 ? row0_valid : row1_valid;
+          const bool ok_r = !valid_row || r[rr] == neg_inf ||
+                            (m_true[rr] != neg_inf && (r[rr] - m_true[rr]) < p.log2_lambda);
+          row_ok = row_ok && ok_r;
+        }
+        skip = __all_sync(0xffffffffu, row_ok) != 0;
+        if (!skip) {
+          m_true[0] = fmaxf(m_true[0], r[0]);
+          m_true[1] = fmaxf(m_true[1], r[1]);
+        }
+        if (p.skip_mask && warp == 0 && lane == 0)
+          p.skip_mask[(size_t(seq) * p.Hkv + kvh) * p.max_tiles + t0 / kDecTile] = skip ? 1 : 0;
+      }
 
-        // ---- S = q K^T for this warp's 16 tokens (two 8-token column tiles)
-        float s[2][4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-        {
-          const int mi = lane >> 3, r = lane & 7;
-          const int tok = tok_base + (mi >> 1) * 8 + r;
-#pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kaddr + swz_off(tok, ks * 2 + (mi & 1)), b0, b1, b2, b3);
-            mma_bf16_16816(s[0], qa[ks], b0, b1);
-            mma_bf16_16816(s[1], qa[ks], b2, b3);
+      if (!skip) {
+        // zero the V rows of masked tokens so that 0 * (stale or NaN) cannot reach O
+        if (!tile_clean) {
+          bool any_masked = false;
+          for (int t = 0; t < 16; ++t) {
+            const int tok = tok_base + t;
+            const bool masked = tok >= ntok || ((bad >> (tok / p.chunk)) & 1u);
+            any_masked |= masked;
+            if (masked) {
+              for (int c = lane; c < D / 8; c += 32)
+                *reinterpret_cast<uint4*>(smem + slot * L::kStageBytes + L::kTileBytes + swz_off<D>(tok, c)) =
+                    make_uint4(0, 0, 0, 0);
+            }
           }
+          if (any_masked) __syncwarp();
         }
-        // ---- scale to log2 units and mask tokens past the end or in invalid pages
-        const bool tile_clean = (ntok == kDecTile) && (bad == 0);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int tok = tok_base + j * 8 + 2 * tq + (e & 1);
-            float v = s[j][e] * p.scale_log2;
-            if (!tile_clean && (tok >= ntok || ((bad >> (tok / p.chunk)) & 1u))) v = neg_inf;
-            s[j][e] = v;
-          }
-        }
-        // warp-local tile row maxima (rows g, g + 8)
-        float mx[2];
-        mx[0] = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-        mx[1] = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+        // reference maximum: raised only when the tile exceeds it by more than 2^8
+        float alpha[2] = {1.f, 1.f};
+        bool raised = false;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+          if (mx[r] != neg_inf && (m_ref[r] == neg_inf || mx[r] > m_ref[r] + kDecRescaleThreshold)) {
+            alpha[r] = (m_ref[r] == neg_inf) ? 0.f : fast_exp2(m_ref[r] - mx[r]);
+            m_ref[r] = mx[r];
+            raised = true;
+          }
         }
-
-        bool skip = false;
-        if constexpr (SKIP) {
-          // tile row maxima over all four warps, then the unit-wide decision
-          if (tq == 0) {
-            red[(red_par * kDecConsumerWarps + warp) * 16 + g] = mx[0];
-            red[(red_par * kDecConsumerWarps + warp) * 16 + g + 8] = mx[1];
-          }
-          named_bar_sync(1, kDecConsumerWarps * 32);
-          float r[2] = {neg_inf, neg_inf};
+        if (__any_sync(0xffffffffu, raised)) {
 #pragma unroll
-          for (int w = 0; w < kDecConsumerWarps; ++w) {
-            r[0] = fmaxf(r[0], red[(red_par * kDecConsumerWarps + w) * 16 + g]);
-            r[1] = fmaxf(r[1], red[(red_par * kDecConsumerWarps + w) * 16 + g + 8]);
+          for (int n = 0; n < NT; ++n) {
+            o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
+            o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
           }
-          red_par ^= 1;
-          bool row_ok = true;
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const bool valid_row = rr == 0 ? row0_valid : row1_valid;
-            const bool ok_r = !valid_row || r[rr] == neg_inf ||
-                              (m_true[rr] != neg_inf && (r[rr] - m_true[rr]) < p.log2_lambda);
-            row_ok = row_ok && ok_r;
-          }
-          skip = __all_sync(0xffffffffu, row_ok) != 0;
-          if (!skip) {
-            m_true[0] = fmaxf(m_true[0], r[0]);
-            m_true[1] = fmaxf(m_true[1], r[1]);
-          }
-          if (p.skip_mask && warp == 0 && lane == 0)
-            p.skip_mask[(size_t(seq) * p.Hkv + kvh) * p.max_tiles + t0 / kDecTile] = skip ? 1 : 0;
+          l_part[0] *= alpha[0];
+          l_part[1] *= alpha[1];
         }
-
-        if (!skip) {
-          // zero the V rows of masked tokens so that 0 * (stale or NaN) cannot reach O
-          if (!tile_clean) {
-            bool any_masked = false;
-            for (int t = 0; t < 16; ++t) {
-              const int tok = tok_base + t;
-              const bool masked = tok >= ntok || ((bad >> (tok / p.chunk)) & 1u);
-              any_masked |= masked;
-              if (masked) {
-                for (int c = lane; c < D / 8; c += 32)
-                  *reinterpret_cast<uint4*>(smem + slot * L::kStageBytes + L::kTileBytes + swz_off(tok, c)) =
-                      make_uint4(0, 0, 0, 0);
-              }
-            }
-            if (any_masked) __syncwarp();
-          }
-          // reference maximum: raised only when the tile exceeds it by more than 2^8
-          float alpha[2] = {1.f, 1.f};
-          bool raised = false;
+        // probabilities, packed as the A operand of P V
+        uint32_t pa[4];
+        {
+          const float off0 = m_ref[0] == neg_inf ? 0.f : m_ref[0];
+          const float off1 = m_ref[1] == neg_inf ? 0.f : m_ref[1];
+          float pr[2][4];
 #pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            if (mx[r] != neg_inf && (m_ref[r] == neg_inf || mx[r] > m_ref[r] + kDecRescaleThreshold)) {
-              alpha[r] = (m_ref[r] == neg_inf) ? 0.f : fast_exp2(m_ref[r] - mx[r]);
-              m_ref[r] = mx[r];
-              raised = true;
-            }
+          for (int j = 0; j < 2; ++j) {
+            pr[j][0] = row0_valid ? fast_exp2(s[j][0] - off0) : 0.f;
+            pr[j][1] = row0_valid ? fast_exp2(s[j][1] - off0) : 0.f;
+            pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
+            pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
           }
-          if (__any_sync(0xffffffffu, raised)) {
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
-              o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
-            }
-            l_part[0] *= alpha[0];
-            l_part[1] *= alpha[1];
-          }
-          // probabilities, packed as the A operand of P V
-          uint32_t pa[4];
-          {
-            const float off0 = m_ref[0] == neg_inf ? 0.f : m_ref[0];
-            const float off1 = m_ref[1] == neg_inf ? 0.f : m_ref[1];
-            float pr[2][4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              pr[j][0] = row0_valid ? fast_exp2(s[j][0] - off0) : 0.f;
-              pr[j][1] = row0_valid ? fast_exp2(s[j][1] - off0) : 0.f;
-              pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
-              pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
-            }
-            l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-            l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
-            pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-            pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-            pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-            pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
-          }
-          // ---- O += P V over this warp's 16 tokens
-          {
-            const int mi = lane >> 3, r = lane & 7;
-            const int tok = tok_base + (mi & 1) * 8 + r;
-#pragma unroll
-            for (int n2 = 0; n2 < NT / 2; ++n2) {
-              uint32_t v0, v1, v2, v3;
-              ldsm_x4_t(vaddr + swz_off(tok, n2 * 2 + (mi >> 1)), v0, v1, v2, v3);
-              mma_bf16_16816(o[2 * n2], pa, v0, v1);
-              mma_bf16_16816(o[2 * n2 + 1], pa, v2, v3);
-            }
-          }
-          if (!tile_clean) fence_proxy_async_smem();  // zeroed rows before the next TMA write
+          l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+          l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+          pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+          pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+          pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+          pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
-        if (++slot == NS) { slot = 0; phase ^= 1u; }
+        // ---- O += P V over this warp's 16 tokens
+        {
+          const int mi = lane >> 3, r = lane & 7;
+          const int tok = tok_base + (mi & 1) * 8 + r;
+#pragma unroll
+          for (int n2 = 0; n2 < NT / 2; ++n2) {
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_t(vaddr + swz_off<D>(tok, n2 * 2 + (mi >> 1)), v0, v1, v2, v3);
+            mma_bf16_16816(o[2 * n2], pa, v0, v1);
+            mma_bf16_16816(o[2 * n2 + 1], pa, v2, v3);
+          }
+        }
+        if (!tile_clean) fence_proxy_async_smem();  // zeroed rows before the next TMA write
       }
-      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+
+      if (++slot == NS) { slot = 0; phase ^= 1u; }
+      if (!last_tile) continue;
 
       // ---- merge the four warps' (m, l, O) in a fixed order and write the split result
 #pragma unroll
@@ -453,6 +526,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           }
         }
       }
+      // the next item's partials overwrite comb_* only after its first tile's
+      // per-warp work; order those writes after every thread's reads above
+      named_bar_sync(1, kDecConsumerWarps * 32);
     }
   }
   __syncwarp();

@@ -1,0 +1,371 @@
+// Dense paged decode with one CTA item per group of KV heads.
+//
+// Work item = (split, sequence, group of HG KV heads), handed out in that
+// order (largest splits first) by an atomic ticket counter in the workspace,
+// which the host zeroes before the launch. A stage is 16 tokens of the item:
+// one TMA copy brings the K rows of all HG heads (a contiguous 16-token x HG-head
+// block of a page) and one the V rows; the tensor map orders heads outside
+// tokens, so each head's 16 rows land as one 4 KB (D = 128) 128-byte-swizzled
+// block. The producer warp reads the next item's length and first block-table
+// window one item ahead and ships each item's query rows with its first stage.
+//
+// Consumer warp h owns KV head h of the group: per stage it computes its G query
+// heads' scores for the 16 tokens and P.V with mma.m16n8k16 (rows >= G zero),
+// runs the online softmax in its accumulator registers across the whole item,
+// and writes the item's result for its heads at the end -- no cross-warp merge.
+// Split partials are combined by decode_merge_kernel as in the per-head path.
+#pragma once
+
+#include "decode.cuh"
+
+namespace attn {
+
+constexpr int kDhChunk = 16;  // tokens per stage
+
+template <int D, int G, int HG>
+struct DecodeHeadsSmem {
+  static constexpr int kHeadBytes = kDhChunk * D * 2;   // one head's 16 tokens
+  static constexpr int kKVBytes = HG * kHeadBytes;      // K (or V) rows of one stage
+  static constexpr int kQBytes = HG * G * D * 2;        // the item's query rows
+  static constexpr int kStageBytes = (2 * kKVBytes + kQBytes + 1023) / 1024 * 1024;
+  static constexpr int kFit = (232448 - 2048) / (kStageBytes + 48);
+  static constexpr int kStages = kFit < 8 ? kFit : 8;
+  static constexpr int kRing = kStages * kStageBytes;
+  static constexpr int kFull = kRing;
+  static constexpr int kEmpty = kFull + 8 * kStages;
+  static constexpr int kInfo = kEmpty + 8 * kStages;   // TileInfo per stage
+  static constexpr int kTotal = kInfo + 32 * kStages;
+  static constexpr int kDynamic = kTotal + 1024;
+  static_assert(kDynamic <= 232448, "shared memory per block");
+  static_assert(kStages >= 2, "ring depth");
+};
+
+// item -> (split, seq, group): splits outermost so that full-length splits go first
+__device__ __forceinline__ void dh_item_coords(long long item, int num_seqs, int n_groups, int& seq, int& split,
+                                               int& grp) {
+  const long long per = (long long)num_seqs * n_groups;
+  split = int(item / per);
+  const int rem = int(item % per);
+  seq = rem / n_groups;
+  grp = rem % n_groups;
+}
+
+template <int D, int G, int HG>
+__global__ void __launch_bounds__((HG + 1) * 32, 1)
+    decode_heads_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const DecodeParams p, int* ticket_counter) {
+  static_assert(G >= 1 && G <= 16, "query heads per KV head");
+  using L = DecodeHeadsSmem<D, G, HG>;
+  constexpr int NS = L::kStages;
+  constexpr int KS = D / 16;
+  constexpr int NT = D / 8;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kFull);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::kEmpty);
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + L::kInfo);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int capacity = p.max_pages * p.page_size;
+  const int n_groups = p.Hkv / HG;
+  const long long num_items = (long long)p.max_splits * p.num_seqs * n_groups;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], HG);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == HG) {
+    // ------------------------------------------------------------ producer warp
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    int slot = 0;
+    uint32_t phase = 0;
+    uint32_t pending = 0, pending_phase = 0;
+    bool ok = true;
+    // next item (ticket), its length and first block-table window, one item ahead
+    long long nx_item = 0;
+    int nx_len = 0, nx_win = -1;
+    auto fetch_next = [&]() {
+      long long t = 0;
+      if (lane == 0) t = atomicAdd(ticket_counter, 1);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      nx_item = t;
+      if (t < num_items) {
+        int sq, sp, gr;
+        dh_item_coords(t, p.num_seqs, n_groups, sq, sp, gr);
+        nx_len = __ldg(&p.seq_lens[sq]);
+        const int e = (((sp * p.split_tokens) / p.page_size) & ~31) + lane;
+        nx_win = e < p.max_pages ? __ldg(&p.block_table[size_t(sq) * p.max_pages + e]) : -1;
+      }
+    };
+    fetch_next();
+    while (ok) {
+      const long long item = nx_item;
+      if (item >= num_items) break;
+      int len = nx_len;
+      int win_cur = nx_win;
+      fetch_next();
+      int seq, split, grp;
+      dh_item_coords(item, p.num_seqs, n_groups, seq, split, grp);
+      if (len > capacity || len < 0) {
+        if (lane == 0 && split == 0 && grp == 0) raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
+        len = len < 0 ? 0 : capacity;
+      }
+      const int t_begin = split * p.split_tokens;
+      if (t_begin >= len) continue;
+      const int t_end = min(t_begin + p.split_tokens, len);
+      const int32_t* bt_row = p.block_table + size_t(seq) * p.max_pages;
+      int win = (t_begin / p.page_size) >> 5;
+      int win_next;
+      {
+        const int e = (win + 1) * 32 + lane;
+        win_next = e < p.max_pages ? __ldg(&bt_row[e]) : -1;
+      }
+      const __nv_bfloat16* qsrc = p.q + (size_t(seq) * p.Hq + size_t(grp) * HG * G) * D;
+      for (int t0 = t_begin; t0 < t_end && ok; t0 += kDhChunk) {
+        const int e0 = t0 / p.page_size;
+        if ((e0 >> 5) != win) {
+          win = e0 >> 5;
+          win_cur = win_next;
+          const int e = (win + 1) * 32 + lane;
+          win_next = e < p.max_pages ? __ldg(&bt_row[e]) : -1;
+        }
+        if (!mbar_wait(&empty[slot], phase ^ 1u, &abort_flag, p.status)) { ok = false; break; }
+        const int page = __shfl_sync(0xffffffffu, win_cur, e0 & 31);
+        if (lane == 0) {
+          const bool valid = page >= 0 && page < p.num_pages;
+          if (!valid) raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
+          const bool first = t0 == t_begin;
+          TileInfo ti;
+          ti.seq = seq; ti.split = split; ti.kvh = grp; ti.t0 = t0;
+          ti.ntok = min(kDhChunk, len - t0);
+          ti.bad = valid ? 0 : 1;
+          ti.flags = (first ? 1 : 0) | (t0 + kDhChunk >= t_end ? 2 : 0);
+          ti.len = len;
+          info[slot] = ti;
+          uint8_t* stage = smem + slot * L::kStageBytes;
+          mbar_arrive_expect_tx(&full[slot], (valid ? uint32_t(2 * L::kKVBytes) : 0u) + (first ? uint32_t(L::kQBytes) : 0u));
+          if (first) bulk_load(stage + 2 * L::kKVBytes, qsrc, uint32_t(L::kQBytes), &full[slot]);
+          if (valid) {
+            const int in_page = t0 % p.page_size;
+            tma_load_5d(stage, &tm_k, &full[slot], 0, 0, in_page, grp * HG, page);
+            tma_load_5d(stage + L::kKVBytes, &tm_v, &full[slot], 0, 0, in_page, grp * HG, page);
+          }
+        }
+        __syncwarp();
+        pending |= 1u << slot;
+        pending_phase = (pending_phase & ~(1u << slot)) | (phase << slot);
+        if (++slot == NS) { slot = 0; phase ^= 1u; }
+      }
+    }
+    if (ok && mbar_wait(&empty[slot], phase ^ 1u, &abort_flag, p.status)) {
+      if (lane == 0) {  // end-of-work marker: a stage with no copies
+        TileInfo ti{};
+        ti.flags = 4;
+        info[slot] = ti;
+        mbar_arrive_expect_tx(&full[slot], 0u);
+      }
+      __syncwarp();
+    } else {
+      ok = false;
+    }
+    if (!ok && lane == 0) {
+      for (int s = 0; s < NS; ++s)
+        if (pending & (1u << s)) mbar_drain(&full[s], (pending_phase >> s) & 1u);
+    }
+  } else {
+    // ------------------------------------------------------------ consumer warp = KV head `warp` of the group
+    const float neg_inf = -__int_as_float(0x7f800000);
+    const int g = lane >> 2, tq = lane & 3;
+    const bool row0_valid = g < G, row1_valid = g + 8 < G;
+    int slot = 0;
+    uint32_t phase = 0;
+    int no_abort = 0;
+    bool ok = true;
+    const uint32_t ring_addr = smem_u32(smem);
+    int seq = 0, split = 0, grp = 0, n_splits = 0;
+    uint32_t qa[KS][4];
+    float o[NT][4];
+    float m_ref[2] = {neg_inf, neg_inf};
+    float l_part[2] = {0.f, 0.f};
+
+    while (ok) {
+      if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) { ok = false; break; }
+      const TileInfo ti = info[slot];
+      if (ti.flags & 4) break;
+      uint8_t* stage = smem + slot * L::kStageBytes;
+      if (ti.flags & 1) {
+        seq = ti.seq; split = ti.split; grp = ti.kvh;
+        n_splits = (ti.len + p.split_tokens - 1) / p.split_tokens;
+        const uint32_t* qs = reinterpret_cast<const uint32_t*>(stage + 2 * L::kKVBytes) + warp * G * (D / 2);
+        const int h0 = row0_valid ? g : 0, h1 = row1_valid ? g + 8 : 0;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qa[ks][0] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + tq] : 0u;
+          qa[ks][1] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + tq] : 0u;
+          qa[ks][2] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + 4 + tq] : 0u;
+          qa[ks][3] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + 4 + tq] : 0u;
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+        m_ref[0] = m_ref[1] = neg_inf;
+        l_part[0] = l_part[1] = 0.f;
+      }
+      const bool last = (ti.flags & 2) != 0;
+      if (!ti.bad) {
+        const int ntok = ti.ntok;
+        const uint32_t kaddr = ring_addr + slot * L::kStageBytes + warp * L::kHeadBytes;
+        const uint32_t vaddr = kaddr + L::kKVBytes;
+        // ---- S = q K^T (16 tokens = two 8-token column tiles; k-steps alternate accumulators)
+        float s[2][4];
+        {
+          float sp[2][2][4];
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int a = 0; a < 2; ++a) sp[j][a][0] = sp[j][a][1] = sp[j][a][2] = sp[j][a][3] = 0.f;
+          const int mi = lane >> 3, r = lane & 7;
+          const int tok = (mi >> 1) * 8 + r;
+          uint32_t bfr[KS][4];
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks)
+            ldsm_x4(kaddr + swz_off<D>(tok, ks * 2 + (mi & 1)), bfr[ks][0], bfr[ks][1], bfr[ks][2], bfr[ks][3]);
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            mma_bf16_16816(sp[0][ks & 1], qa[ks], bfr[ks][0], bfr[ks][1]);
+            mma_bf16_16816(sp[1][ks & 1], qa[ks], bfr[ks][2], bfr[ks][3]);
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[j][e] = sp[j][0][e] + sp[j][1][e];
+        }
+        const bool clean = ntok == kDhChunk;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tok = j * 8 + 2 * tq + (e & 1);
+            const float v = s[j][e] * p.scale_log2;
+            s[j][e] = (!clean && tok >= ntok) ? neg_inf : v;
+          }
+        float mx[2];
+        mx[0] = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        mx[1] = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        }
+        if (!clean) {
+          // zero the V rows of tokens past the end so that 0 * (stale or NaN) cannot reach O
+          for (int t = ntok; t < kDhChunk; ++t)
+            for (int c = lane; c < D / 8; c += 32)
+              *reinterpret_cast<uint4*>(stage + L::kKVBytes + warp * L::kHeadBytes + swz_off<D>(t, c)) =
+                  make_uint4(0, 0, 0, 0);
+          __syncwarp();
+        }
+        float alpha[2] = {1.f, 1.f};
+        bool raised = false;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          if (mx[r] != neg_inf && (m_ref[r] == neg_inf || mx[r] > m_ref[r] + kDecRescaleThreshold)) {
+            alpha[r] = (m_ref[r] == neg_inf) ? 0.f : fast_exp2(m_ref[r] - mx[r]);
+            m_ref[r] = mx[r];
+            raised = true;
+          }
+        }
+        if (__any_sync(0xffffffffu, raised)) {
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
+            o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
+          }
+          l_part[0] *= alpha[0];
+          l_part[1] *= alpha[1];
+        }
+        uint32_t pa[4];
+        {
+          const float off0 = m_ref[0] == neg_inf ? 0.f : m_ref[0];
+          const float off1 = m_ref[1] == neg_inf ? 0.f : m_ref[1];
+          float pr[2][4];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            pr[j][0] = row0_valid ? fast_exp2(s[j][0] - off0) : 0.f;
+            pr[j][1] = row0_valid ? fast_exp2(s[j][1] - off0) : 0.f;
+            pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
+            pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
+          }
+          l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+          l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+          pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+          pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+          pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+          pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+        }
+        // ---- O += P V over the 16 tokens
+        {
+          const int mi = lane >> 3, r = lane & 7;
+          const int tok = (mi & 1) * 8 + r;
+#pragma unroll
+          for (int n2 = 0; n2 < NT / 2; ++n2) {
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_t(vaddr + swz_off<D>(tok, n2 * 2 + (mi >> 1)), v0, v1, v2, v3);
+            mma_bf16_16816(o[2 * n2], pa, v0, v1);
+            mma_bf16_16816(o[2 * n2 + 1], pa, v2, v3);
+          }
+        }
+        if (!clean) fence_proxy_async_smem();   // zeroed rows before the next TMA write
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (++slot == NS) { slot = 0; phase ^= 1u; }
+      if (!last) continue;
+
+      // ---- the item's result for this warp's G query heads
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 1);
+        l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 2);
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const bool valid = r == 0 ? row0_valid : row1_valid;
+        if (!valid) continue;
+        const int hq = (grp * HG + warp) * G + g + 8 * r;
+        const float lsum = l_part[r];
+        const float inv = lsum > 0.f ? 1.f / lsum : 0.f;   // 0 only if every page was invalid
+        if (n_splits == 1) {
+          __nv_bfloat16* dst = p.o + (size_t(seq) * p.Hq + hq) * D + 2 * tq;
+#pragma unroll
+          for (int n = 0; n < NT; ++n)
+            *reinterpret_cast<uint32_t*>(dst + n * 8) = pack_bf16x2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+          if (p.lse && tq == 0)
+            p.lse[size_t(seq) * p.Hq + hq] = lsum > 0.f ? (m_ref[r] + __log2f(lsum)) * 0.69314718055994531f : neg_inf;
+        } else {
+          float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + 2 * tq;
+#pragma unroll
+          for (int n = 0; n < NT; ++n)
+            *reinterpret_cast<float2*>(dst + n * 8) = make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+          if (tq == 0)
+            p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lsum > 0.f ? m_ref[r] + __log2f(lsum) : neg_inf;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+}
+
+}  // namespace attn

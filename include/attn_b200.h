@@ -40,6 +40,7 @@
  *     (out-of-range block-table entries, a pipeline wait that timed out) are
  *     reported through `device_status` when given, and always through the
  *     library's device status word (attn_read_device_status). No kernel traps.
+ *     The status words keep the largest code recorded.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -105,8 +106,9 @@ int attn_prefill_blasst(const void* q, const void* k, const void* v, void* o, fl
  * attn_decode_workspace_bytes -- scratch needed by attn_decode_paged.
  * The decode splits each sequence's keys into chunks of split_tokens tokens,
  * computes one partial (O, LSE) per (sequence, query head, chunk), and merges
- * them. The workspace holds those partials:
- *   fp32 [num_seqs][max_splits][Hq][D] + fp32 [num_seqs][max_splits][Hq]
+ * them. The workspace holds a 256-byte header (the kernel's work counter,
+ * reset by the library on every call) and those partials:
+ *   fp32 [num_seqs][max_splits][Hq][D] (padded to 256 B) + fp32 [num_seqs][max_splits][Hq]
  * with max_splits = ceil(max_pages_per_seq * page_size / split_tokens).
  * Returns 0 for invalid arguments.
  */
@@ -189,7 +191,8 @@ int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_
 /*
  * attn_read_device_status -- read (and, if clear != 0, reset to ATTN_OK) the
  * library's device status word on the current device. Synchronises the
- * device. Every kernel of the library ORs a device-side error into it.
+ * device. Every kernel of the library records device-side errors in it (the
+ * largest code wins).
  */
 int attn_read_device_status(int* status_out, int clear);
 

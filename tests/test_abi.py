@@ -74,11 +74,12 @@ def test_prefill_blasst_rejects_bad_lambda(lib):
 
 
 def test_workspace_bytes(lib):
-    # fp32 [N][splits][Hq][D] padded to 256 B, then fp32 [N][splits][Hq]
+    # a 256 B header (work-ticket counter), fp32 [N][splits][Hq][D] padded to 256 B,
+    # then fp32 [N][splits][Hq]
     n, hq, d, mp, ps, sp = 64, 32, 128, 512, 16, 1024
     splits = -(-mp * ps // sp)
     o_bytes = n * splits * hq * d * 4
-    want = -(-o_bytes // 256) * 256 + n * splits * hq * 4
+    want = 256 + -(-o_bytes // 256) * 256 + n * splits * hq * 4
     assert lib.attn_decode_workspace_bytes(n, hq, d, mp, ps, sp) == want
     assert ab.decode_workspace_bytes(n, hq, d, mp, ps, sp) == want
     for bad in [(0, hq, d, mp, ps, sp), (n, hq, 96, mp, ps, sp), (n, hq, d, mp, 24, sp), (n, hq, d, mp, ps, 100),
