@@ -150,7 +150,9 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.n_qblocks = (S + 2 * kPfRows - 1) / (2 * kPfRows);
   p.n_qt = (S + kPfRows - 1) / kPfRows;
   p.n_kt = (S + 63) / 64;
-  p.num_items = (long long)p.n_qblocks * B * Hq;
+  const long long num_items = (long long)p.n_qblocks * B * Hq;
+  if (num_items > 0x7fffffffll) return ATTN_ERR_UNSUPPORTED;
+  p.num_items = int(num_items);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.log2_lambda = lambda > 0.f ? std::log2(lambda) : -INFINITY;
 

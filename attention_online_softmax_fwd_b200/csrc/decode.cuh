@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     float o[NT][4];
     float m_ref[2] = {neg_inf, neg_inf};   // per-warp exponent reference, rows g and g + 8
     float m_true[2] = {neg_inf, neg_inf};  // unit's running max of kept tiles (tile skip)
-    float l_part[2] = {0.f, 0.f};          // this lane's share of the row sums
+    float l_part[2] = {0.f, 0.f};          // this lane's share of the row sums (-> LSE)
+    float lr_part[2] = {0.f, 0.f};         // the same as rounded to bf16 for P V (-> normalises O)
 
     while (ok) {
       if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) {
@@ -311,6 +312,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         m_ref[0] = m_ref[1] = neg_inf;
         m_true[0] = m_true[1] = neg_inf;
         l_part[0] = l_part[1] = 0.f;
+        lr_part[0] = lr_part[1] = 0.f;
       }
       const bool last_tile = (ti.flags & 2) != 0;
       const uint32_t kaddr = ring_addr + slot * L::kStageBytes;
@@ -431,6 +433,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           }
           l_part[0] *= alpha[0];
           l_part[1] *= alpha[1];
+          lr_part[0] *= alpha[0];
+          lr_part[1] *= alpha[1];
         }
         // probabilities, packed as the A operand of P V
         uint32_t pa[4];
@@ -445,12 +449,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
             pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
           }
-          l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-          l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
           pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
           pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
           pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
           pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+          l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+          l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+          // the weights applied to V are normalised by the sum of the rounded P, so
+          // they add up to one (a dominant key's P, up to 2^8 under the lagging
+          // reference, would otherwise carry its bf16 rounding into the whole row)
+          lr_part[0] += (bf16_lo(pa[0]) + bf16_hi(pa[0])) + (bf16_lo(pa[2]) + bf16_hi(pa[2]));
+          lr_part[1] += (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));
         }
         // ---- O += P V over this warp's 16 tokens
         {
@@ -477,13 +486,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       for (int r = 0; r < 2; ++r) {
         l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 1);
         l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 2);
+        lr_part[r] += __shfl_xor_sync(0xffffffffu, lr_part[r], 1);
+        lr_part[r] += __shfl_xor_sync(0xffffffffu, lr_part[r], 2);
       }
+      const float inv_r0 = lr_part[0] > 0.f ? 1.f / lr_part[0] : 0.f;
+      const float inv_r1 = lr_part[1] > 0.f ? 1.f / lr_part[1] : 0.f;
       if (row0_valid) {
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           float* dst = comb_o + (warp * G + g) * D + n * 8 + 2 * tq;
-          dst[0] = o[n][0];
-          dst[1] = o[n][1];
+          dst[0] = o[n][0] * inv_r0;
+          dst[1] = o[n][1] * inv_r0;
         }
         if (tq == 0) { comb_m[warp * G + g] = m_ref[0]; comb_l[warp * G + g] = l_part[0]; }
       }
@@ -491,8 +504,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           float* dst = comb_o + (warp * G + g + 8) * D + n * 8 + 2 * tq;
-          dst[0] = o[n][2];
-          dst[1] = o[n][3];
+          dst[0] = o[n][2] * inv_r1;
+          dst[1] = o[n][3] * inv_r1;
         }
         if (tq == 0) { comb_m[warp * G + g + 8] = m_ref[1]; comb_l[warp * G + g + 8] = l_part[1]; }
       }
@@ -508,8 +521,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         for (int w = 0; w < kDecConsumerWarps; ++w) {
           const float mw = comb_m[w * G + h];
           const float e = (mw == neg_inf) ? 0.f : fast_exp2(mw - M);
-          lsum += e * comb_l[w * G + h];
-          osum += e * comb_o[(w * G + h) * D + d];
+          const float wl = e * comb_l[w * G + h];
+          lsum += wl;
+          osum += wl * comb_o[(w * G + h) * D + d];   // comb_o holds each warp's normalised partial
         }
         const float val = lsum > 0.f ? osum / lsum : 0.f;  // 0 only if every page was invalid
         const int hq = kvh * G + h;

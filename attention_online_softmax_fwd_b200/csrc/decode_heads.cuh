@@ -198,7 +198,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     uint32_t qa[KS][4];
     float o[NT][4];
     float m_ref[2] = {neg_inf, neg_inf};
-    float l_part[2] = {0.f, 0.f};
+    float l_part[2] = {0.f, 0.f};    // row sums of the probabilities (-> LSE)
+    float lr_part[2] = {0.f, 0.f};   // the same as rounded to bf16 for P V (-> normalises O)
 
     while (ok) {
       if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) { ok = false; break; }
@@ -221,6 +222,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
         m_ref[0] = m_ref[1] = neg_inf;
         l_part[0] = l_part[1] = 0.f;
+        lr_part[0] = lr_part[1] = 0.f;
       }
       const bool last = (ti.flags & 2) != 0;
       if (!ti.bad) {
@@ -294,6 +296,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           }
           l_part[0] *= alpha[0];
           l_part[1] *= alpha[1];
+          lr_part[0] *= alpha[0];
+          lr_part[1] *= alpha[1];
         }
         uint32_t pa[4];
         {
@@ -307,12 +311,17 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
             pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
             pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
           }
-          l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-          l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
           pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
           pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
           pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
           pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+          l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+          l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+          // the weights applied to V are normalised by the sum of the rounded P, so
+          // they add up to one (a dominant key's P, up to 2^8 under the lagging
+          // reference, would otherwise carry its bf16 rounding into the whole row)
+          lr_part[0] += (bf16_lo(pa[0]) + bf16_hi(pa[0])) + (bf16_lo(pa[2]) + bf16_hi(pa[2]));
+          lr_part[1] += (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));
         }
         // ---- O += P V over the 16 tokens
         {
@@ -338,6 +347,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       for (int r = 0; r < 2; ++r) {
         l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 1);
         l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 2);
+        lr_part[r] += __shfl_xor_sync(0xffffffffu, lr_part[r], 1);
+        lr_part[r] += __shfl_xor_sync(0xffffffffu, lr_part[r], 2);
       }
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
@@ -345,7 +356,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         if (!valid) continue;
         const int hq = (grp * HG + warp) * G + g + 8 * r;
         const float lsum = l_part[r];
-        const float inv = lsum > 0.f ? 1.f / lsum : 0.f;   // 0 only if every page was invalid
+        const float inv = lr_part[r] > 0.f ? 1.f / lr_part[r] : 0.f;   // 0 only if every page was invalid
         if (n_splits == 1) {
           __nv_bfloat16* dst = p.o + (size_t(seq) * p.Hq + hq) * D + 2 * tq;
 #pragma unroll

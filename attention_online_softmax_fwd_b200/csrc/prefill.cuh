@@ -3,21 +3,28 @@
 //
 // A persistent CTA walks work items (b, hq, 256-row query block), longest
 // causal blocks first. The query block is two 128-row tiles, A and B, that
-// share every K/V tile the CTA loads. Roles (384 threads):
+// share every K/V tile the CTA loads. Roles (384 threads, 12 warps):
 //   warp 0      TMA producer: Q_A, Q_B once per item, then K_0, K_1, V_0,
 //               K_2, V_1, ... into a ring (each K one tile ahead of its V)
 //   warps 1, 2  MMA issuers, one thread per query tile; warp 1 owns the TMEM allocation
+//   warp 3      idle (it only gives up registers)
 //   warps 4-7   softmax of tile A (thread t <-> row t <-> TMEM lane t)
 //   warps 8-11  softmax of tile B
+// Each of the four SM sub-partitions holds warps w, w + 4, w + 8 (one of warps
+// 0-3 and one warp of each softmax warpgroup) and owns a quarter of the
+// register file, so the register split is balanced within every sub-partition.
 // Tensor memory (512 columns): S_A | S_B | O_A | O_B, fp32.
 // Per KV tile j the issuer of tile X issues S_X(j+1) = Q_X K_{j+1}^T as soon as
 // the softmax of tile X has copied S_X(j) into registers, and O_X += P_X(j) V_j
 // once the softmax has written the bf16 probabilities P_X(j) to shared
-// memory; the two tiles' issuers never wait on each other's softmax. So the exponentials of tile j overlap the next tile's Q K^T, and
-// the tensor pipe has queued work while either softmax warpgroup computes.
+// memory; the two tiles' issuers never wait on each other's softmax. So the
+// exponentials of tile j overlap the next tile's Q K^T, and the tensor pipe has
+// queued work while either softmax warpgroup computes.
 // The exponentials use a reference maximum that is only raised when the tile
-// maximum exceeds it by more than 2^8 (exact: O and l share the reference);
-// the BLASST decisions use the true running maximum of the kept tiles.
+// maximum exceeds it by more than 2^8 (exact: O and l share the reference).
+// BLASST tile skip: each softmax warp publishes a vote per 64-key half and the
+// MMA issuer combines the four; a warp waits for the others only when its own
+// rows would drop the whole tile (then it does no exponentials at all).
 #pragma once
 
 #include "common.cuh"
@@ -32,7 +39,7 @@ struct PrefillParams {
   int B, S, Hq, Hkv;
   int n_qblocks;       // ceil(S / 256)
   int n_qt, n_kt;      // ceil(S / 128), ceil(S / 64)
-  long long num_items;
+  int num_items;       // n_qblocks * B * Hq (< 2^31)
   float scale_log2;    // scale * log2(e)
   float log2_lambda;   // log2(lambda) (tile skip only)
 };
@@ -40,10 +47,14 @@ struct PrefillParams {
 constexpr int kPfRows = 128;     // rows per query tile
 constexpr int kPfKeys = 128;     // keys per K/V tile (two 64-key decision tiles)
 constexpr int kPfThreads = 384;
+constexpr int kPfProducerWarp = 0, kPfIssuerWarp0 = 1;   // issuer of tile x: warp 1 + x
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// setmaxnreg split: warps 0-3 drop to 96 registers, warps 4-11 rise to 200.
-constexpr int kPfRegsLow = 96, kPfRegsHigh = 200;
+// setmaxnreg split: warps 0-3 drop to kPfRegsLow registers, the softmax warps rise to
+// kPfRegsHigh. Per sub-partition: low + 2 * high <= 3 * 168, the launch allocation.
+constexpr int kPfRegsLow = 72, kPfRegsHigh = 216;
 constexpr int kPfRegPoolNeeded = 128 * kPfRegsLow + 256 * kPfRegsHigh;  // must fit the launch allocation
+constexpr int kPfLaunchRegs = 168;   // 168 x 384 = 64512
+static_assert(kPfRegsLow + 2 * kPfRegsHigh <= 3 * kPfLaunchRegs, "register split exceeds a sub-partition's share");
 
 template <int D>
 struct PrefillSmem {
@@ -58,8 +69,10 @@ struct PrefillSmem {
   // barrier indices (pairs are per query tile)
   static constexpr int bQFull = 0, bQEmpty = 2, bSFull = 4, bSFree = 6, bPFull = 8, bPVDone = 10, bOEmpty = 12,
                        bTeardown = 14, bKVFull = 15, bKVEmpty = 15 + kStages, kNumBars = 15 + 2 * kStages;
-  static constexpr int kMisc = kBars + 8 * kNumBars;            // tmem base, flags, votes
+  static constexpr int kMisc = kBars + 8 * kNumBars;            // tmem base, flags
+  static constexpr int kVotes = (kMisc + 16 + 15) / 16 * 16;    // skip votes [2][4][4] ints
   static constexpr int kTotal = kMisc + 256;
+  static_assert(kVotes + 128 <= kTotal, "skip votes exceed the misc area");
   static constexpr int kDynamic = kTotal + 1024;
 };
 
@@ -82,14 +95,118 @@ __device__ __forceinline__ void pf_issue_qk(uint32_t d_tmem, uint64_t qdesc, uin
 
 // O (+)= P V: P K-major (keys contiguous) and V MN-major, both from shared
 // memory; 8 MMAs of 128 x D x 16 keys. 16 keys = 32 B of a P row and 2 KB of V.
+// Bit h of skip_halves leaves out the four MMAs of 64-key half h.
 template <int D>
-__device__ __forceinline__ void pf_issue_pv(uint32_t d_tmem, uint64_t pdesc, uint64_t vdesc, bool accumulate) {
+__device__ __forceinline__ void pf_issue_pv(uint32_t d_tmem, uint64_t pdesc, uint64_t vdesc, bool accumulate,
+                                            int skip_halves) {
   constexpr uint32_t idesc = make_idesc_bf16(128, D, 0, 1);
+  bool acc = accumulate;
 #pragma unroll
   for (int kk = 0; kk < kPfKeys / 16; ++kk) {
+    if ((skip_halves >> (kk / 4)) & 1) continue;
     const uint64_t poff16 = uint64_t(((kk / 4) * (kPfRows * 128) + (kk % 4) * 32) >> 4);
-    umma_ss(d_tmem, pdesc + poff16, vdesc + uint64_t((kk * 16 * 128) >> 4), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
+    umma_ss(d_tmem, pdesc + poff16, vdesc + uint64_t((kk * 16 * 128) >> 4), idesc, acc ? 1u : 0u);
+    acc = true;
+  }
+}
+
+// Tile-wide skip decision of one query tile and one K/V tile: the AND of the
+// four softmax warps' votes (bit h set: every row of the warp lets 64-key half h
+// go). A vote word is (tag << 2) | bits, the tag naming the tile in the
+// warpgroup's sequence, so a stale word is never taken for a fresh one. The
+// four words of a tile are adjacent and 16-byte aligned.
+__device__ __forceinline__ int4 pf_votes_v4(const volatile int* words) {
+  int4 w;
+  asm volatile("ld.volatile.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+               : "r"(smem_u32(const_cast<const int*>(words)))
+               : "memory");
+  return w;
+}
+__device__ __forceinline__ bool pf_votes_all_in(const int4& w, int tag) {
+  return ((w.x >> 2) == tag) & ((w.y >> 2) == tag) & ((w.z >> 2) == tag) & ((w.w >> 2) == tag);
+}
+
+// Waits (bounded by the pipeline wait limit) for all four votes; -1 on timeout.
+// Kept out of line: it runs only when a vote is late, and inlined it would
+// crowd the registers of the softmax loop.
+__device__ __forceinline__ int pf_tile_decision_wait(const volatile int* words, int tag, volatile int* abort_flag,
+                                                  int* user_status) {
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    const int4 w = pf_votes_v4(words);
+    if (pf_votes_all_in(w, tag)) return w.x & w.y & w.z & w.w & 3;
+    if ((i & 31u) == 0) {
+      if (*abort_flag) return -1;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        raise_status(user_status, ATTN_ERR_TIMEOUT);
+        return -1;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int pf_tile_decision(const volatile int* words, int tag, volatile int* abort_flag,
+                                                int* user_status) {
+  const int4 w = pf_votes_v4(words);
+  if (pf_votes_all_in(w, tag)) return w.x & w.y & w.z & w.w & 3;
+  return pf_tile_decision_wait(words, tag, abort_flag, user_status);
+}
+
+// Row-sum pairs (exact, as rounded for P V), added and scaled without contraction.
+__device__ __forceinline__ float2 sum2_add(float2 a, float2 b) {
+  return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
+}
+__device__ __forceinline__ float2 sum2_scale(float2 a, float s) {
+  return make_float2(__fmul_rn(a.x, s), __fmul_rn(a.y, s));
+}
+// The sums of the 64-key halves that decision d keeps (bit h: half h skipped).
+__device__ __forceinline__ float2 sum2_kept(const float2 (&h)[2], int d) {
+  const float2 a = (d & 1) ? make_float2(0.f, 0.f) : h[0];
+  const float2 b = (d & 2) ? make_float2(0.f, 0.f) : h[1];
+  return make_float2(a.x + b.x, a.y + b.y);
+}
+
+// This thread's row of S from tensor memory (128 columns), with keys past the
+// causal diagonal or the sequence end set to -inf.
+template <bool CAUSAL>
+__device__ __forceinline__ void pf_load_scores(uint32_t taddr, float (&s)[kPfKeys], int key0, int row, int row0,
+                                               int S) {
+  uint32_t sr[kPfKeys];
+  ATTN_TMEM_LD32_NOWAIT(taddr + 0, sr + 0);
+  ATTN_TMEM_LD32_NOWAIT(taddr + 32, sr + 32);
+  ATTN_TMEM_LD32_NOWAIT(taddr + 64, sr + 64);
+  ATTN_TMEM_LD32_NOWAIT(taddr + 96, sr + 96);
+  tmem_ld_wait();
+  ATTN_REG_FENCE32(sr + 0);
+  ATTN_REG_FENCE32(sr + 32);
+  ATTN_REG_FENCE32(sr + 64);
+  ATTN_REG_FENCE32(sr + 96);
+#pragma unroll
+  for (int e = 0; e < kPfKeys; ++e) s[e] = __uint_as_float(sr[e]);
+  const float neg_inf = -__int_as_float(0x7f800000);
+  const bool full_tile = (!CAUSAL || key0 + kPfKeys - 1 <= row0) && (key0 + kPfKeys <= S);
+  if (!full_tile) {
+#pragma unroll
+    for (int e = 0; e < kPfKeys; ++e) {
+      const int key = key0 + e;
+      if ((CAUSAL && key > row) || key >= S) s[e] = neg_inf;
+    }
+  }
+}
+
+// Record the decisions for K/V tile jt (two 64-key tiles) of query tile qt:
+// 1 skipped, 0 kept; tiles past the causal diagonal or the sequence stay untouched.
+template <bool CAUSAL>
+__device__ __forceinline__ void pf_write_skip_mask(const PrefillParams& p, int b, int hq, int qt, int jt,
+                                                   int last_row, int decision) {
+  uint8_t* mrow = p.skip_mask + ((size_t(b) * p.Hq + hq) * p.n_qt + qt) * p.n_kt;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k64 = jt * kPfKeys + h * 64;
+    const bool visited = k64 < p.S && (!CAUSAL || k64 <= last_row);
+    if (visited) mrow[k64 / 64] = uint8_t((decision >> h) & 1);
   }
 }
 
@@ -106,14 +223,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  volatile int* pv_skip = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);      // [2]
-  volatile int* votes = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);       // [2][4 warps][4]
+  // skip votes [tile x][sequence slot, 4][softmax warp, 4]; slot = tile sequence number mod 4
+  volatile int* votes = reinterpret_cast<volatile int*>(smem + L::kVotes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    for (int i = 0; i < 32; ++i) votes[i] = 0;   // tag 0 never names a tile
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars[L::bQFull + x], 1);
       mbar_init(&bars[L::bQEmpty + x], 1);
@@ -130,7 +248,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kPfIssuerWarp0) {
     tmem_alloc(tmem_base_smem, kTmemCols);
     tmem_relinquish();
   }
@@ -141,10 +259,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   // Item decode shared by all roles: longest causal blocks first; the G query
   // heads of one KV head are adjacent so their K/V tiles are reused from L2.
-  auto item_coords = [&](long long item, int& qb, int& b, int& hq) {
-    const long long per = (long long)p.B * p.Hq;
-    qb = p.n_qblocks - 1 - int(item / per);
-    const int rem = int(item % per);
+  auto item_coords = [&](int item, int& qb, int& b, int& hq) {
+    const int per = p.B * p.Hq;
+    qb = p.n_qblocks - 1 - item / per;
+    const int rem = item % per;
     b = rem / p.Hq;
     hq = rem % p.Hq;
   };
@@ -155,11 +273,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     return (p.S + kPfKeys - 1) / kPfKeys;
   };
 
-  // Register split (launch: 168 x 384 = 64512): warps 0-3 keep kPfRegsLow = 96, the two
-  // softmax warpgroups take kPfRegsHigh = 200 each: 128*96 + 256*200 = 63488 <= 64512.
+  // Register split: warps 0-3 give up registers, the softmax warpgroups take them
+  // (kPfRegPoolNeeded is checked against the launch allocation on the host).
   if (warp < 4) {
     setmaxnreg_dec<kPfRegsLow>();
-    if (warp == 0) {
+    if (warp == kPfProducerWarp) {
       // ============================================================ TMA producer
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
@@ -170,7 +288,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         uint32_t qe_bits = 3u;
         uint32_t pend_mask = 0, pend_ph = 0;
         bool ok = true;
-        for (long long item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+        for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
           int qb, b, hq;
           item_coords(item, qb, b, hq);
           const int kvh = hq / (p.Hq / p.Hkv);
@@ -210,14 +328,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (pend_mask & (1u << s)) mbar_drain(&bars[L::bKVFull + s], (pend_ph >> s) & 1u);
         }
       }
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp == kPfIssuerWarp0 || warp == kPfIssuerWarp0 + 1) {
       // ============================================================ MMA issuers
       // One thread per query tile x (warp 1: A, warp 2: B). Both walk the whole
       // K/V ring of every item and arrive on each slot's empty barrier (count 2),
       // whether or not their tile uses the slot; an issuer never runs more than
       // one ring phase ahead because it waits for each slot's load first.
       if (lane == 0) {
-        const int x = warp - 1;
+        const int x = warp - kPfIssuerWarp0;
         const uint32_t q_desc_addr = smem_u32(smem + L::kQ + x * L::kTileBytes);
         const uint32_t p_desc_addr = smem_u32(smem + L::kP + x * L::kPBytes);
         const uint32_t ring_addr = smem_u32(smem + L::kRing);
@@ -226,9 +344,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         uint32_t phase = 0;
         uint32_t qf_ph = 0u, sfree_ph = 0u, pf_ph = 0u, oe_ph = 1u;
         bool qk_started = false;  // a Q K^T has been issued for this tile in this kernel
+        int seq = 0;              // P V tiles of this query tile so far (skip-vote sequence)
         bool ok = true;
 
-        for (long long item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+        for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
           int qb, b, hq;
           item_coords(item, qb, b, hq);
           const int rows0 = tile_rows(qb, 0), rows1 = tile_rows(qb, 1);
@@ -266,8 +385,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!mbar_wait(&bars[L::bPFull + x], pf_ph, abort_flag, p.status)) { ok = false; break; }
               pf_ph ^= 1u;
               tc_fence_after();
-              const bool skip_pv = SKIP && pv_skip[x] != 0;
-              if (!skip_pv) {
+              int skip_halves = 0;
+              if constexpr (SKIP) {
+                // every softmax warp voted before arriving on P_full
+                ++seq;
+                skip_halves = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, abort_flag, p.status);
+                if (skip_halves < 0) { ok = false; break; }
+              }
+              if (skip_halves != 3) {
                 if (!pv_started) {
                   // first P V of this item: the previous item's epilogue must have read O_x
                   if (!mbar_wait(&bars[L::bOEmpty + x], oe_ph, abort_flag, p.status)) { ok = false; break; }
@@ -275,7 +400,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                   tc_fence_after();
                 }
                 pf_issue_pv<D>(d_o, make_sdesc_sw128(p_desc_addr, 16, 1024),
-                               make_sdesc_sw128(ring_addr + cur * L::kTileBytes, L::kChunkBytes, 1024), pv_started);
+                               make_sdesc_sw128(ring_addr + cur * L::kTileBytes, L::kChunkBytes, 1024), pv_started,
+                               skip_halves);
                 pv_started = true;
               }
               umma_commit(&bars[L::bPVDone + x]);   // P_x free; after the last tile: O_x final
@@ -303,9 +429,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int own_timeout_only = 0;
     volatile int* no_abort = reinterpret_cast<volatile int*>(&own_timeout_only);
     uint32_t sf_ph = 0, pvd_ph = 0;
+    int seq = 0;   // K/V tiles of this query tile so far (skip-vote sequence)
     bool ok = true;
 
-    for (long long item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+    for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
       int qb, b, hq;
       item_coords(item, qb, b, hq);
       const int rows = tile_rows(qb, x);
@@ -315,38 +442,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int row = row0 + t;
       const bool row_valid = t < rows;
       const int last_row = row0 + rows - 1;
-      float m_ref = neg_inf, m_true = neg_inf, l = 0.f;
+      float m_ref = neg_inf, m_true = neg_inf;
+      // Row sums at the reference m_ref: .x sums the probabilities (-> LSE); .y
+      // normalises O and differs from .x by the bf16 rounding of each half's largest
+      // probability: under the lagging reference a dominant key has P up to 2^8, and
+      // its rounding, left out of the sum, would scale the whole output row.
+      float2 l = make_float2(0.f, 0.f);
 
       for (int j = 0; j < nkv; ++j) {
         if (!mbar_wait(&bars[L::bSFull + x], sf_ph, no_abort, p.status)) { ok = false; break; }
         sf_ph ^= 1u;
         tc_fence_after();
-        uint32_t sr[kPfKeys];
-        ATTN_TMEM_LD32_NOWAIT(taddr_s + 0, sr + 0);
-        ATTN_TMEM_LD32_NOWAIT(taddr_s + 32, sr + 32);
-        ATTN_TMEM_LD32_NOWAIT(taddr_s + 64, sr + 64);
-        ATTN_TMEM_LD32_NOWAIT(taddr_s + 96, sr + 96);
-        tmem_ld_wait();
-        ATTN_REG_FENCE32(sr + 0);
-        ATTN_REG_FENCE32(sr + 32);
-        ATTN_REG_FENCE32(sr + 64);
-        ATTN_REG_FENCE32(sr + 96);
-        // S_x is in registers: the tensor pipe may overwrite it with the next tile
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[L::bSFree + x]);
-
-        float s[kPfKeys];
-#pragma unroll
-        for (int e = 0; e < kPfKeys; ++e) s[e] = __uint_as_float(sr[e]);
         const int key0 = j * kPfKeys;
-        const bool full_tile = (!CAUSAL || key0 + kPfKeys - 1 <= row0) && (key0 + kPfKeys <= p.S);
-        if (!full_tile) {
-#pragma unroll
-          for (int e = 0; e < kPfKeys; ++e) {
-            const int key = key0 + e;
-            if ((CAUSAL && key > row) || key >= p.S) s[e] = neg_inf;
-          }
+        float s[kPfKeys];
+        pf_load_scores<CAUSAL>(taddr_s, s, key0, row, row0, p.S);
+        if constexpr (!SKIP) {
+          // S_x is in registers: the tensor pipe may overwrite it with the next tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[L::bSFree + x]);
         }
         // row maxima of the two 64-key halves (raw scores; scale > 0 commutes with max)
         float mx[2];
@@ -370,82 +484,90 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) r2[h] = (mx[h] == neg_inf) ? neg_inf : mx[h] * p.scale_log2;
 
-        bool skip_h[2] = {false, false};
+        // Tile skip (SKIP only): this warp's vote, bit h set when every one of its
+        // rows lets 64-key half h go. The running maximum used by the test takes
+        // in every visited score: a half that is skipped lies below it by
+        // -log2(lambda) > 0, so this equals the maximum over kept halves.
+        // A warp that keeps a half does not wait for the other votes: it computes
+        // the exponentials at once. That is exact whatever the outcome, since a
+        // skipped half can neither raise the reference maximum (it lies below the
+        // running maximum, which is within 2^8 of the reference) nor set it when
+        // it is raised. The issuer leaves skipped halves out of P V, and the row
+        // sums of the kept halves are added to l once P is handed over.
+        // A warp that would drop the whole tile waits for the tile-wide decision
+        // with S still in tensor memory (S_free not yet given), so the scores
+        // need not stay in registers meanwhile; it reloads them if the tile is kept.
+        int vote = 0, decision = -1;
+        bool skip_all = false;
         if constexpr (SKIP) {
-          // Decisions for both 64-key halves with one barrier: half 1 is voted
-          // under both outcomes of half 0.
-          auto row_ok = [&](float r, float m) {
-            return !row_valid || r == neg_inf || (m != neg_inf && (r - m) < p.log2_lambda);
-          };
-          const bool ok0 = row_ok(r2[0], m_true);
-          const bool ok1_if_skip0 = row_ok(r2[1], m_true);
-          const bool ok1_if_keep0 = row_ok(r2[1], fmaxf(m_true, r2[0]));
-          const int v0 = __all_sync(0xffffffffu, ok0);
-          const int v1 = __all_sync(0xffffffffu, ok1_if_skip0);
-          const int v2 = __all_sync(0xffffffffu, ok1_if_keep0);
-          volatile int* my_votes = votes + (x * 4 + wq) * 4;
-          if (lane == 0) { my_votes[0] = v0; my_votes[1] = v1; my_votes[2] = v2; }
-          named_bar_sync(1 + x, 128);
-          int a0 = 1, a1 = 1, a2 = 1;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            a0 &= votes[(x * 4 + w) * 4 + 0];
-            a1 &= votes[(x * 4 + w) * 4 + 1];
-            a2 &= votes[(x * 4 + w) * 4 + 2];
+          const float lam2 = p.log2_lambda;
+          const bool ok0 = !row_valid || r2[0] == neg_inf || (m_true != neg_inf && r2[0] - m_true < lam2);
+          const float m1 = fmaxf(m_true, r2[0]);
+          const bool ok1 = !row_valid || r2[1] == neg_inf || (m1 != neg_inf && r2[1] - m1 < lam2);
+          m_true = fmaxf(m1, r2[1]);
+          vote = (__all_sync(0xffffffffu, ok0) ? 1 : 0) | (__all_sync(0xffffffffu, ok1) ? 2 : 0);
+          ++seq;
+          if (lane == 0) votes[x * 16 + (seq & 3) * 4 + wq] = (seq << 2) | vote;
+          if (vote == 3) {
+            decision = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status);
+            if (decision < 0) { ok = false; break; }
+            skip_all = decision == 3;
+            if (!skip_all) pf_load_scores<CAUSAL>(taddr_s, s, key0, row, row0, p.S);
           }
-          skip_h[0] = a0 != 0;
-          skip_h[1] = skip_h[0] ? (a1 != 0) : (a2 != 0);
-          if (!skip_h[0]) m_true = fmaxf(m_true, r2[0]);
-          if (!skip_h[1]) m_true = fmaxf(m_true, r2[1]);
-          if (p.skip_mask && t == 0) {
-            const int qt = qb * 2 + x;
-            uint8_t* mrow = p.skip_mask + ((size_t(b) * p.Hq + hq) * p.n_qt + qt) * p.n_kt;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int k64 = key0 + h * 64;
-              const bool visited = k64 < p.S && (!CAUSAL || k64 <= last_row);
-              if (visited) mrow[k64 / 64] = skip_h[h] ? 1 : 0;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[L::bSFree + x]);
+          if (skip_all) {
+            // the whole tile is dropped: no exponentials, no P, no P V (l, O and
+            // the reference stay as they are); keep the P V phase count in step
+            if (j > 0) {
+              if (!mbar_wait(&bars[L::bPVDone + x], pvd_ph, no_abort, p.status)) { ok = false; break; }
+              pvd_ph ^= 1u;
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[L::bPFull + x]);
+            if (p.skip_mask && t == 0) pf_write_skip_mask<CAUSAL>(p, b, hq, qb * 2 + x, j, last_row, 3);
+            continue;
           }
         }
-        const bool skip_all = skip_h[0] && skip_h[1];
         uint32_t pk[kPfKeys / 2];   // this row's probabilities, bf16 pairs
         float alpha = 1.f;
         bool raise = false;
-        if (!skip_all) {
-          float m_tile = neg_inf;
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            if (!skip_h[h]) m_tile = fmaxf(m_tile, r2[h]);
+        float2 hsum[2];   // the halves' row sums
+        {
+          const float m_tile = fmaxf(r2[0], r2[1]);
           // raise the reference maximum only when needed (or on the first finite tile)
           raise = (m_tile != neg_inf) && (m_ref == neg_inf || m_tile > m_ref + kRescaleThreshold);
           if (raise) {
             alpha = (m_ref == neg_inf) ? 0.f : fast_exp2(m_ref - m_tile);
             m_ref = m_tile;
-            l *= alpha;
           }
           const float offset = (m_ref == neg_inf) ? 0.f : m_ref;
           const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
           const uint64_t negoff2 = f2_pack(-offset, -offset);
-          uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+          uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
           for (int e = 0; e < kPfKeys / 2; ++e) {
-            if (skip_h[e / 32]) {
-              pk[e] = 0u;
-            } else {
-              const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), scale2, negoff2);
-              float x0, x1;
-              f2_unpack(xx, x0, x1);
-              const float p0 = fast_exp2(x0);
-              const float p1 = fast_exp2(x1);
-              sum2[e & 1] = f2_add(sum2[e & 1], f2_pack(p0, p1));
-              pk[e] = pack_bf16x2(p0, p1);
-            }
+            const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), scale2, negoff2);
+            float x0, x1;
+            f2_unpack(xx, x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            pk[e] = pack_bf16x2(p0, p1);
+            sum2[(e / 32) * 2 + (e & 1)] = f2_add(sum2[(e / 32) * 2 + (e & 1)], f2_pack(p0, p1));
           }
-          float sa, sb, sc, sd;
-          f2_unpack(sum2[0], sa, sb);
-          f2_unpack(sum2[1], sc, sd);
-          l += (sa + sb) + (sc + sd);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float sa, sb, sc, sd;
+            f2_unpack(sum2[2 * h], sa, sb);
+            f2_unpack(sum2[2 * h + 1], sc, sd);
+            hsum[h].x = (sa + sb) + (sc + sd);
+            // The normalising sum takes the largest probability of the half as
+            // rounded for P V (the same fma and exp2 as in the loop above give the
+            // same value): that term dominates the rounding error of the weights
+            // (P up to 2^8 under the lagging reference), the others average out.
+            const float pm = fast_exp2(fmaf(mx[h], p.scale_log2, -offset));
+            hsum[h].y = (mx[h] == neg_inf) ? hsum[h].x : hsum[h].x + (bf16_lo(pack_bf16x2(pm, pm)) - pm);
+          }
         }
         // P_x(j-1) must have been consumed (and O_x updated) before P_x(j) is written
         // and before any rescale of O_x; the exponentials above overlapped that P V.
@@ -454,7 +576,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           pvd_ph ^= 1u;
           tc_fence_after();
         }
-        if (!skip_all) {
+        // l <- l * alpha + (kept halves' sums), without contraction so that lambda = 0
+        // through the skip path rounds exactly like the dense path
+        l = sum2_scale(l, alpha);
+        if constexpr (!SKIP) l = sum2_add(l, sum2_kept(hsum, 0));
+        {
           if (__any_sync(0xffffffffu, raise && j > 0)) {
             // rescale this warp's rows of O (every P V of earlier tiles has completed)
 #pragma unroll
@@ -477,9 +603,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           fence_proxy_async_smem();   // the tensor pipe reads P through the async proxy
         }
         tc_fence_before();
-        if (t == 0) pv_skip[x] = skip_all ? 1 : 0;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[L::bPFull + x]);
+        if constexpr (SKIP) {
+          // The other warps voted before their exponentials, so by now the
+          // decision is normally complete; fold in the sums of the kept halves.
+          const int d = decision >= 0 ? decision : pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status);
+          if (d < 0) { ok = false; break; }
+          l = sum2_add(l, sum2_kept(hsum, d));
+          if (p.skip_mask && t == 0) pf_write_skip_mask<CAUSAL>(p, b, hq, qb * 2 + x, j, last_row, d);
+        }
       }
       if (!ok) break;
 
@@ -487,7 +620,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!mbar_wait(&bars[L::bPVDone + x], pvd_ph, no_abort, p.status)) { ok = false; break; }
       pvd_ph ^= 1u;
       tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_l = (l.y > 0.f) ? 1.f / l.y : 0.f;
       __nv_bfloat16* orow = p.o + ((size_t(b) * p.S + row) * p.Hq + hq) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -506,7 +639,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       if (row_valid && p.lse)
         p.lse[(size_t(b) * p.Hq + hq) * p.S + row] =
-            (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : neg_inf;
+            (l.x > 0.f) ? (m_ref + __log2f(l.x)) * 0.69314718055994531f : neg_inf;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[L::bOEmpty + x]);
@@ -517,7 +650,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kPfIssuerWarp0) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace attn

@@ -351,7 +351,7 @@ def run_gpu(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel<128,causal>", "achieved": pre_tfs,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": pre_tfs / peaks["bf16_tflops"],
                      "peak_source": f"{peak_src} bf16 burst", "traffic": traffic.get("prefill_bytes_per_launch")},
-        "roofline_decode": {"bound": "hbm", "kernel": "decode_split_kernel<128,4>+decode_merge_kernel",
+        "roofline_decode": {"bound": "hbm", "kernel": "decode_heads_kernel<128,4,8>+decode_merge_kernel",
                             "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": dec_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy",
                             "traffic": traffic.get("decode_bytes_per_call")},
@@ -364,12 +364,70 @@ def run_gpu(args, world, rank, local):
         "wall_s_timed_region": wall,
         "outputs_finite": finite,
     }
+    if rank == 0 and world == 1 and not args.no_blasst:
+        line["blasst_long_context"] = blasst_long_context_report(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfs, gbs, secs, desc = oracle_sample(int(args.cpu_heads), 4)
         line["cpu_baseline"] = {"value": tfs, "unit": "TFLOP/s", "cores": cpu_threads()[0], "kind": "oracle",
                                 "sample": desc, "decode_gbs": gbs, "seconds": secs}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def blasst_long_context_report(dev, reps=3):
+    """Long-context BLASST workload (B=1, Hq=32, Hkv=8, S=32768, D=128, 64-key tiles):
+    prefill and the decode of the last row at lambda in {0, 0.1, 0.3}. Reports the
+    time, the skipped fraction of visited tiles and the error against lambda = 0."""
+    import attention_online_softmax_fwd_b200 as ab
+    c = gen.CONFIGS["blasst_long_context"]
+    B, Hq, Hkv, S, D = c["B"], c["Hq"], c["Hkv"], c["S"], c["D"]
+    q_h, k_h, v_h = gen.peaked_prefill_inputs(B, Hq, Hkv, S, D, c["seed"], amp=4.0, period=64)
+    cache = gen.paged_from_contiguous(q_h[:, S - 1], k_h, v_h, page_size=c["page_size"], seed=c["seed"] + 1,
+                                      poison=False)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    dargs = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    scale = gen.attn_scale(D)
+    split = 256   # 128 splits of the one sequence: enough work items for every SM
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            out = fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts), out
+
+    fl = prefill_flops(B, Hq, S, D)
+    dbytes = decode_bytes([S], Hq, Hkv, D, cache.max_pages)
+    report = {"workload": "blasst_long_context B1 Hq32 Hkv8 S32768 D128, tiles of 64 keys, decode split 256",
+              "prefill": {}, "decode": {}}
+    ms0, (o0, l0) = timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale))
+    dms0, (do0, dl0) = timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=split))
+    report["prefill"]["0.0"] = {"ms": ms0, "tflops": fl / (ms0 * 1e-3) / 1e12, "skipped_frac": 0.0}
+    report["decode"]["0.0"] = {"ms": dms0, "gbs": dbytes / (dms0 * 1e-3) / 1e9, "skipped_frac": 0.0}
+    for lam in (0.1, 0.3):
+        ms, (o, l, mask) = timed(lambda: ab.prefill_blasst(q, k, v, lam, causal=True, scale=scale))
+        vis = (mask != 2)
+        err = (o.float() - o0.float()).abs()
+        report["prefill"][str(lam)] = {
+            "ms": ms, "tflops_dense_equiv": fl / (ms * 1e-3) / 1e12,
+            "skipped_frac": float(((mask == 1) & vis).sum().item() / vis.sum().item()),
+            "max_abs_err_vs_dense": float(err.max().item()), "mean_abs_err_vs_dense": float(err.mean().item()),
+            "speedup_vs_dense": ms0 / ms}
+        dms, (do, dl, dmask) = timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split))
+        dvis = (dmask != 2)
+        derr = (do.float() - do0.float()).abs()
+        report["decode"][str(lam)] = {
+            "ms": dms, "gbs_dense_equiv": dbytes / (dms * 1e-3) / 1e9,
+            "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
+            "max_abs_err_vs_dense": float(derr.max().item()), "speedup_vs_dense": dms0 / dms}
+    return report
 
 
 def main():
@@ -379,6 +437,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-blasst", action="store_true", help="skip the long-context BLASST report")
     ap.add_argument("--cpu-heads", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3:

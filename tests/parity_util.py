@@ -69,3 +69,20 @@ def compare_skip(mask_gpu, mask_ref, margin_ref, label=""):
     assert not hard.any(), f"{label}: {int(hard.sum())} skip decisions differ outside the tie band"
     return {"decisions": int(visited_ref.sum()), "skipped": int((mr == 1).sum()),
             "tie_mismatches": int((diff & ties).sum())}
+
+
+def assert_rounding_limited(o_gpu, o_ref, ulps=0.6, floor=2e-4, label=""):
+    """Every element within ``ulps`` bf16 spacings of the exact value (plus ``floor``).
+
+    Rounding the exact result to bf16 costs at most half a spacing; the rest of
+    the budget covers the fp32 arithmetic. An error in the normalisation of a
+    row (such as the bf16 rounding of one dominant probability left out of l)
+    scales the whole row and shows up here long before the absolute bound.
+    """
+    og = o_gpu.detach().float().cpu().double().numpy() if isinstance(o_gpu, torch.Tensor) else np.asarray(o_gpu)
+    orf = np.asarray(o_ref, dtype=np.float64)
+    err = np.abs(og - orf)
+    bound = ulps * bf16_ulp(orf) + floor
+    bad = err > bound
+    assert not bad.any(), (f"{label}: {int(bad.sum())} elements beyond {ulps} bf16 spacing "
+                           f"(worst {float((err / bf16_ulp(orf)).max()):.2f} spacings)")

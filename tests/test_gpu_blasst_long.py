@@ -1,0 +1,77 @@
+"""Long-context BLASST workload (B=1, Hq=32, Hkv=8, S=32768, D=128, 64-key
+tiles, lambda in {0, 0.1, 0.3}; Q and every 64th key carry 4u for a seeded unit
+vector u): prefill and the decode of the last row over the paged cache, on the
+GPU against the float64 oracle on sampled decision units and rows."""
+
+import numpy as np
+import pytest
+import torch
+
+import attention_online_softmax_fwd_b200 as ab
+from attention_online_softmax_fwd_b200 import inputs as gen
+from oracle import attn_oracle as orc
+from parity_util import compare_output, compare_skip
+
+pytestmark = pytest.mark.gpu
+
+C = gen.CONFIGS["blasst_long_context"]
+SPLIT = 2048
+
+
+@pytest.fixture(scope="module")
+def workload():
+    q, k, v = gen.peaked_prefill_inputs(C["B"], C["Hq"], C["Hkv"], C["S"], C["D"], C["seed"], amp=4.0, period=64)
+    cache = gen.paged_from_contiguous(q[:, C["S"] - 1], k, v, page_size=C["page_size"], seed=C["seed"] + 1)
+    return q, k, v, cache
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.1, 0.3])
+def test_long_context_prefill(cuda_device, workload, lam):
+    q, k, v, _ = workload
+    dev = cuda_device
+    scale = gen.attn_scale(C["D"])
+    o, lse, mask = ab.prefill_blasst(q.to(dev), k.to(dev), v.to(dev), lam, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    heads = [(0, 3), (0, 30)]
+    q_tiles = [0, 77, 255]
+    o_ref, lse_ref, m_ref, margin = orc.prefill_blasst(q, k, v, True, scale, lam, heads=heads, q_tiles=q_tiles)
+    mg = mask.cpu().numpy()
+    og, lg = o.cpu(), lse.cpu()
+    for b, h in heads:
+        for qt in q_tiles:
+            st = compare_skip(mg[b, h, qt], m_ref[b, h, qt], margin[b, h, qt], label=f"h={h} qt={qt}")
+            rows = list(range(qt * 128, qt * 128 + 128))
+            if st["tie_mismatches"] == 0:
+                compare_output(og[b, rows, h], o_ref[b, rows, h], lg[b, h, rows], lse_ref[b, h, rows],
+                               label=f"lam={lam} h={h} qt={qt}")
+    if lam == 0.0:
+        assert not (mask == 1).any()
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.1, 0.3])
+def test_long_context_decode(cuda_device, workload, lam):
+    q, k, v, cache = workload
+    dev = cuda_device
+    scale = gen.attn_scale(C["D"])
+    args = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    o, lse, mask = ab.decode_paged_blasst(*args, lam, scale=scale, split_tokens=SPLIT)
+    torch.cuda.synchronize()
+    o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages,
+                                                            cache.block_table, cache.seq_lens, C["page_size"],
+                                                            scale, lam, SPLIT)
+    st = compare_skip(mask, m_ref, margin, label=f"decode lam={lam}")
+    if st["tie_mismatches"] == 0:
+        compare_output(o, o_ref, lse, lse_ref, label=f"decode lam={lam}")
+    print(f"decode lam={lam}: skipped {st['skipped']} of {st['decisions']} tiles")
+
+
+def test_long_context_decode_equals_prefill_last_row(cuda_device, workload):
+    q, k, v, cache = workload
+    dev = cuda_device
+    scale = gen.attn_scale(C["D"])
+    o, lse = ab.prefill(q.to(dev), k.to(dev), v.to(dev), causal=True, scale=scale)
+    od, ld = ab.decode_paged(*[t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table,
+                                                   cache.seq_lens)], scale=scale, split_tokens=SPLIT)
+    torch.cuda.synchronize()
+    S = C["S"]
+    compare_output(od[0], o[0, S - 1].float().cpu().double().numpy(), ld[0], lse[0, :, S - 1].cpu().numpy())

@@ -7,7 +7,7 @@ import torch
 import attention_online_softmax_fwd_b200 as ab
 from attention_online_softmax_fwd_b200 import inputs as gen
 from oracle import attn_oracle as orc
-from parity_util import compare_output, compare_skip
+from parity_util import assert_rounding_limited, compare_output, compare_skip
 
 pytestmark = pytest.mark.gpu
 
@@ -77,6 +77,24 @@ def test_decode_blasst_matches_oracle(cuda_device, split, lam):
     assert st["skipped"] > 0
     if st["tie_mismatches"] == 0:
         compare_output(o, o_ref, lse, lse_ref, label=f"decode blasst lam={lam}")
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 2)])
+def test_decode_dominant_key_normalisation(cuda_device, Hq, Hkv):
+    # a dominant key at 0 and a stronger one at 200 (P = 2^7.3 under the lagging
+    # reference): the output must stay within rounding of the exact value
+    S, D = 3000, 128
+    q, k, v = gen.peaked_prefill_inputs(1, Hq, Hkv, S, D, seed=2250, amp=12.0, period=1 << 30)
+    k[:, 200] = (k[:, 0].float() * 1.4).to(torch.bfloat16)
+    cache = gen.paged_from_contiguous(q[:, S - 1], k, v, page_size=16, seed=2251)
+    for split in (256, 4096):
+        o, lse, _, scale = _run(cache, cuda_device, split)
+        o_ref, lse_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens,
+                                          16, scale)
+        compare_output(o, o_ref, lse, lse_ref, label=f"dominant key split={split}")
+        assert_rounding_limited(o, o_ref, label=f"dominant key split={split}")
+        o, lse, _, _ = _run(cache, cuda_device, split, 0.0)   # the per-KV-head kernel
+        assert_rounding_limited(o, o_ref, label=f"dominant key lambda 0 split={split}")
 
 
 def test_decode_lambda_zero_mask_is_dense(cuda_device):

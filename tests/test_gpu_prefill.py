@@ -7,7 +7,7 @@ import torch
 import attention_online_softmax_fwd_b200 as ab
 from attention_online_softmax_fwd_b200 import inputs as gen
 from oracle import attn_oracle as orc
-from parity_util import compare_output, compare_skip
+from parity_util import assert_rounding_limited, compare_output, compare_skip
 
 pytestmark = pytest.mark.gpu
 
@@ -87,6 +87,46 @@ def test_prefill_blasst_matches_oracle(cuda_device, causal):
         if st["tie_mismatches"] == 0:
             compare_output(o, o_ref, lse, lse_ref, label=f"prefill blasst lam={lam}")
     assert st["skipped"] > 0
+
+
+def _later_peak_inputs():
+    # one dominant key at 0 and a stronger one at 200: under the lagging reference
+    # maximum the second has P = 2^7.3, which bf16 rounds by up to 2^-8 relative
+    q, k, v = gen.peaked_prefill_inputs(1, 4, 2, 777, 128, seed=3250, amp=12.0, period=1 << 30)
+    k[:, 200] = (k[:, 0].float() * 1.4).to(torch.bfloat16)
+    return q, k, v
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_dominant_key_normalisation(cuda_device, causal):
+    q, k, v = _later_peak_inputs()
+    o, lse, _, scale = _run(q, k, v, causal, cuda_device)
+    o_ref, lse_ref = orc.prefill(q, k, v, causal, scale)
+    assert_rounding_limited(o, o_ref, label=f"dominant key causal={causal}")
+    o, lse, _, scale = _run(q, k, v, causal, cuda_device, 0.01)
+    o_ref, lse_ref, _, _ = orc.prefill_blasst(q, k, v, causal, scale, 0.01)
+    assert_rounding_limited(o, o_ref, label=f"dominant key blasst causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_blasst_later_peak(cuda_device, causal):
+    # a stronger key at 200 (second half of K/V tile 1) after the peak at key 0:
+    # tile 1 keeps its second 64-key half and drops its first, and the running
+    # maximum rises past the first peak
+    q, k, v = _later_peak_inputs()
+    # outputs are close to one row of V; scaled down so that the bf16 rounding of
+    # the output alone stays well inside the mean tolerance
+    v = (v.float() * 0.25).to(torch.bfloat16)
+    kept_second_half_only = 0
+    for lam in (0.01, 0.2):
+        o, lse, mask, scale = _run(q, k, v, causal, cuda_device, lam)
+        o_ref, lse_ref, m_ref, margin = orc.prefill_blasst(q, k, v, causal, scale, lam)
+        st = compare_skip(mask, m_ref, margin, label=f"prefill skip lam={lam}")
+        if st["tie_mismatches"] == 0:
+            compare_output(o, o_ref, lse, lse_ref, label=f"prefill blasst later peak lam={lam}")
+        m = mask.cpu().numpy()
+        kept_second_half_only += int(((m[..., 2] == 1) & (m[..., 3] == 0)).sum())
+    assert kept_second_half_only > 0
 
 
 def test_prefill_lambda_zero_is_dense(cuda_device):
