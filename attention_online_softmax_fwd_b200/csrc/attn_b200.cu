@@ -181,6 +181,14 @@ long long max_splits_of(int max_pages, int page_size, int split_tokens) {
   return (cap + split_tokens - 1) / split_tokens;
 }
 
+// One CTA per (sequence, query head); a no-op for sequences of one split.
+template <int D>
+int launch_merge(const DecodeParams& p, cudaStream_t stream) {
+  const long long pairs = (long long)p.num_seqs * p.Hq;
+  decode_merge_kernel<D><<<dim3(unsigned(pairs)), dim3(kMergeWarps * 32), 0, stream>>>(p);
+  return launch_status();
+}
+
 template <int D, int G, bool SKIP>
 int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int sms,
                   cudaStream_t stream) {
@@ -191,10 +199,7 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodePara
   const long long grid = p.num_items < sms ? p.num_items : sms;
   kernel<<<dim3(unsigned(grid)), dim3(kDecThreads), smem, stream>>>(tk, tv, p);
   if (int st = launch_status()) return st;
-  const long long pairs = (long long)p.num_seqs * p.Hq;
-  const long long blocks = (pairs + 7) / 8;
-  decode_merge_kernel<D><<<dim3(unsigned(blocks)), dim3(256), 0, stream>>>(p);
-  return launch_status();
+  return launch_merge<D>(p, stream);
 }
 
 template <int D, bool SKIP>
@@ -221,9 +226,7 @@ int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
   const long long grid = items < sms ? items : sms;
   kernel<<<dim3(unsigned(grid)), dim3((HG + 1) * 32), smem, stream>>>(tk, tv, p, ticket_counter);
   if (int st = launch_status()) return st;
-  const long long pairs = (long long)p.num_seqs * p.Hq;
-  decode_merge_kernel<D><<<dim3(unsigned((pairs + 7) / 8)), dim3(256), 0, stream>>>(p);
-  return launch_status();
+  return launch_merge<D>(p, stream);
 }
 
 template <int D, int HG>

@@ -549,14 +549,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
 }
 
-// One warp per (sequence, query head): combine the split partials.
+// Combine the split partials of one (sequence, query head) per CTA: each
+// partial is a normalised O row (fp32) with its log2-sum-exp; the result is
+// sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M), M the largest lse_s. The four
+// warps take interleaved splits with several loads in flight, then combine in
+// a fixed order (deterministic).
+constexpr int kMergeWarps = 4;
 template <int D>
-__global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeParams p) {
-  constexpr int DL = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long idx = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (idx >= (long long)p.num_seqs * p.Hq) return;
-  const int seq = int(idx / p.Hq), hq = int(idx % p.Hq);
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const DecodeParams p) {
+  constexpr int DL = D / 32;   // floats per lane: 4 (D = 128) or 2 (D = 64)
+  constexpr int kUnroll = 4;
+  __shared__ float sh_m[kMergeWarps], sh_w[kMergeWarps];
+  __shared__ __align__(16) float sh_acc[kMergeWarps][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq = int(blockIdx.x / unsigned(p.Hq)), hq = int(blockIdx.x % unsigned(p.Hq));
   const int capacity = p.max_pages * p.page_size;
   int len = __ldg(&p.seq_lens[seq]);
   len = len < 0 ? 0 : min(len, capacity);
@@ -565,33 +571,76 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeParams p)
   const float neg_inf = -__int_as_float(0x7f800000);
   if (n_splits == 1) return;  // written by the split kernel
   if (n_splits == 0) {
-#pragma unroll
-    for (int d = 0; d < DL; ++d) orow[lane * DL + d] = __float2bfloat16_rn(0.f);
-    if (p.lse && lane == 0) p.lse[size_t(seq) * p.Hq + hq] = neg_inf;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) orow[d] = __float2bfloat16_rn(0.f);
+    if (p.lse && threadIdx.x == 0) p.lse[size_t(seq) * p.Hq + hq] = neg_inf;
     return;
   }
   const float* lse_base = p.ws_lse + size_t(seq) * p.max_splits * p.Hq + hq;
+  const float* o_base = p.ws_o + (size_t(seq) * p.max_splits * p.Hq + hq) * D + lane * DL;
+  const size_t o_stride = size_t(p.Hq) * D;   // floats between consecutive splits
+  // the largest partial LSE
   float mx = neg_inf;
-  for (int s = lane; s < n_splits; s += 32) mx = fmaxf(mx, lse_base[size_t(s) * p.Hq]);
+  for (int s = threadIdx.x; s < n_splits; s += kMergeWarps * 32) mx = fmaxf(mx, lse_base[size_t(s) * p.Hq]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) sh_m[warp] = mx;
+  __syncthreads();
+  mx = sh_m[0];
+#pragma unroll
+  for (int w = 1; w < kMergeWarps; ++w) mx = fmaxf(mx, sh_m[w]);
+  // this warp's splits: warp, warp + 4, ...
   float acc[DL];
 #pragma unroll
   for (int d = 0; d < DL; ++d) acc[d] = 0.f;
   float wsum = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
+  int s = warp;
+  for (; s + (kUnroll - 1) * kMergeWarps < n_splits; s += kUnroll * kMergeWarps) {
+    float ls[kUnroll], ov[kUnroll][DL];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int su = s + u * kMergeWarps;
+      ls[u] = lse_base[size_t(su) * p.Hq];
+      const float* src = o_base + size_t(su) * o_stride;
+      if constexpr (DL == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(src);
+        ov[u][0] = t.x; ov[u][1] = t.y; ov[u][2] = t.z; ov[u][3] = t.w;
+      } else {
+        const float2 t = *reinterpret_cast<const float2*>(src);
+        ov[u][0] = t.x; ov[u][1] = t.y;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const float w = (ls[u] == neg_inf) ? 0.f : fast_exp2(ls[u] - mx);
+      wsum += w;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) acc[d] = fmaf(w, ov[u][d], acc[d]);
+    }
+  }
+  for (; s < n_splits; s += kMergeWarps) {
     const float ls = lse_base[size_t(s) * p.Hq];
     const float w = (ls == neg_inf) ? 0.f : fast_exp2(ls - mx);
-    const float* orow_s = p.ws_o + ((size_t(seq) * p.max_splits + s) * p.Hq + hq) * D + lane * DL;
+    const float* src = o_base + size_t(s) * o_stride;
     wsum += w;
 #pragma unroll
-    for (int d = 0; d < DL; ++d) acc[d] = fmaf(w, orow_s[d], acc[d]);
+    for (int d = 0; d < DL; ++d) acc[d] = fmaf(w, src[d], acc[d]);
   }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
 #pragma unroll
-  for (int d = 0; d < DL; ++d) orow[lane * DL + d] = __float2bfloat16_rn(acc[d] * inv);
-  if (p.lse && lane == 0)
-    p.lse[size_t(seq) * p.Hq + hq] = wsum > 0.f ? (mx + __log2f(wsum)) * 0.69314718055994531f : neg_inf;
+  for (int d = 0; d < DL; ++d) sh_acc[warp][lane * DL + d] = acc[d];
+  if (lane == 0) sh_w[warp] = wsum;
+  __syncthreads();
+  float wt = sh_w[0];
+#pragma unroll
+  for (int w = 1; w < kMergeWarps; ++w) wt += sh_w[w];
+  const float inv = wt > 0.f ? 1.f / wt : 0.f;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float v = sh_acc[0][d];
+#pragma unroll
+    for (int w = 1; w < kMergeWarps; ++w) v += sh_acc[w][d];
+    orow[d] = __float2bfloat16_rn(v * inv);
+  }
+  if (p.lse && threadIdx.x == 0)
+    p.lse[size_t(seq) * p.Hq + hq] = wt > 0.f ? (mx + __log2f(wt)) * 0.69314718055994531f : neg_inf;
 }
 
 }  // namespace attn

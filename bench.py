@@ -427,6 +427,27 @@ def blasst_long_context_report(dev, reps=3):
             "ms": dms, "gbs_dense_equiv": dbytes / (dms * 1e-3) / 1e9,
             "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
             "max_abs_err_vs_dense": float(derr.max().item()), "speedup_vs_dense": dms0 / dms}
+
+    # The recipe above puts a raised key in every 64-key tile, so no tile can be
+    # dropped. A second input with a single dominant key at position 0 (12 u on
+    # key 0 and on all queries) shows the skip path when most tiles fall below
+    # the running maximum.
+    q_h, k_h, v_h = gen.peaked_prefill_inputs(B, Hq, Hkv, S, D, c["seed"] + 7, amp=12.0, period=S)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    del q_h, k_h, v_h
+    sink = {"input": "12 u on key 0 and on all queries, no other raised keys", "prefill": {}}
+    ms0, (o0, l0) = timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale))
+    sink["prefill"]["0.0"] = {"ms": ms0, "tflops": fl / (ms0 * 1e-3) / 1e12}
+    for lam in (0.1, 0.3):
+        ms, (o, l, mask) = timed(lambda: ab.prefill_blasst(q, k, v, lam, causal=True, scale=scale))
+        vis = (mask != 2)
+        err = (o.float() - o0.float()).abs()
+        sink["prefill"][str(lam)] = {
+            "ms": ms, "tflops_dense_equiv": fl / (ms * 1e-3) / 1e12,
+            "skipped_frac": float(((mask == 1) & vis).sum().item() / vis.sum().item()),
+            "max_abs_err_vs_dense": float(err.max().item()), "mean_abs_err_vs_dense": float(err.mean().item()),
+            "speedup_vs_dense": ms0 / ms}
+    report["dominant_key_input"] = sink
     return report
 
 

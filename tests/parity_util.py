@@ -71,13 +71,16 @@ def compare_skip(mask_gpu, mask_ref, margin_ref, label=""):
             "tie_mismatches": int((diff & ties).sum())}
 
 
-def assert_rounding_limited(o_gpu, o_ref, ulps=0.6, floor=2e-4, label=""):
+def assert_rounding_limited(o_gpu, o_ref, ulps=0.6, floor=1e-3, label=""):
     """Every element within ``ulps`` bf16 spacings of the exact value (plus ``floor``).
 
-    Rounding the exact result to bf16 costs at most half a spacing; the rest of
-    the budget covers the fp32 arithmetic. An error in the normalisation of a
-    row (such as the bf16 rounding of one dominant probability left out of l)
-    scales the whole row and shows up here long before the absolute bound.
+    Rounding the exact result to bf16 costs at most half a spacing; ``floor``
+    covers the bf16 rounding of P where two keys share a row's mass (a weight
+    of 0.05 next to 0.93 moves by ~1e-4 of |v|). An error in the normalisation
+    of a row (such as the bf16 rounding of one dominant probability left out of
+    l) scales the whole row by up to 2^-8 and exceeds this on outputs of order
+    one, where the absolute 1e-2 bound with its one-spacing allowance does not
+    see it.
     """
     og = o_gpu.detach().float().cpu().double().numpy() if isinstance(o_gpu, torch.Tensor) else np.asarray(o_gpu)
     orf = np.asarray(o_ref, dtype=np.float64)

@@ -75,3 +75,55 @@ def test_long_context_decode_equals_prefill_last_row(cuda_device, workload):
     torch.cuda.synchronize()
     S = C["S"]
     compare_output(od[0], o[0, S - 1].float().cpu().double().numpy(), ld[0], lse[0, :, S - 1].cpu().numpy())
+
+
+# Same shapes, one dominant key: 12u on key 0 and on all queries, nothing else
+# raised. Nearly every later tile falls below the running maximum, so this
+# exercises the skip path at ~99% of tiles dropped (the bench's second input).
+@pytest.fixture(scope="module")
+def dominant():
+    q, k, v = gen.peaked_prefill_inputs(C["B"], C["Hq"], C["Hkv"], C["S"], C["D"], C["seed"] + 7, amp=12.0,
+                                        period=C["S"])
+    cache = gen.paged_from_contiguous(q[:, C["S"] - 1], k, v, page_size=C["page_size"], seed=C["seed"] + 8)
+    return q, k, v, cache
+
+
+@pytest.mark.parametrize("lam", [0.1, 0.3])
+def test_long_context_dominant_key_prefill(cuda_device, dominant, lam):
+    q, k, v, _ = dominant
+    dev = cuda_device
+    scale = gen.attn_scale(C["D"])
+    o, lse, mask = ab.prefill_blasst(q.to(dev), k.to(dev), v.to(dev), lam, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    heads = [(0, 5), (0, 17)]
+    q_tiles = [1, 130, 255]
+    o_ref, lse_ref, m_ref, margin = orc.prefill_blasst(q, k, v, True, scale, lam, heads=heads, q_tiles=q_tiles)
+    mg = mask.cpu().numpy()
+    og, lg = o.cpu(), lse.cpu()
+    skipped = 0
+    for b, h in heads:
+        for qt in q_tiles:
+            st = compare_skip(mg[b, h, qt], m_ref[b, h, qt], margin[b, h, qt], label=f"h={h} qt={qt}")
+            skipped += st["skipped"]
+            rows = list(range(qt * 128, qt * 128 + 128))
+            if st["tie_mismatches"] == 0:
+                compare_output(og[b, rows, h], o_ref[b, rows, h], lg[b, h, rows], lse_ref[b, h, rows],
+                               label=f"dominant lam={lam} h={h} qt={qt}")
+    assert skipped > 0.9 * sum(min(2 * qt + 2, C["S"] // 64) for qt in q_tiles) * len(heads)
+
+
+@pytest.mark.parametrize("split", [256, 2048])
+def test_long_context_dominant_key_decode(cuda_device, dominant, split):
+    q, k, v, cache = dominant
+    dev = cuda_device
+    scale = gen.attn_scale(C["D"])
+    args = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    o, lse, mask = ab.decode_paged_blasst(*args, 0.1, scale=scale, split_tokens=split)
+    torch.cuda.synchronize()
+    o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages,
+                                                            cache.block_table, cache.seq_lens, C["page_size"],
+                                                            scale, 0.1, split)
+    st = compare_skip(mask, m_ref, margin, label=f"dominant decode split={split}")
+    assert st["skipped"] > 0
+    if st["tie_mismatches"] == 0:
+        compare_output(o, o_ref, lse, lse_ref, label=f"dominant decode split={split}")

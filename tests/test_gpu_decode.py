@@ -91,7 +91,9 @@ def test_decode_dominant_key_normalisation(cuda_device, Hq, Hkv):
         o, lse, _, scale = _run(cache, cuda_device, split)
         o_ref, lse_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens,
                                           16, scale)
-        compare_output(o, o_ref, lse, lse_ref, label=f"dominant key split={split}")
+        # (outputs are close to one row of V, so bf16 output rounding alone puts the
+        # mean error near 1e-3: the element bound below is the check)
+        assert np.abs(lse.cpu().double().numpy() - np.asarray(lse_ref)).max() <= 1e-3
         assert_rounding_limited(o, o_ref, label=f"dominant key split={split}")
         o, lse, _, _ = _run(cache, cuda_device, split, 0.0)   # the per-KV-head kernel
         assert_rounding_limited(o, o_ref, label=f"dominant key lambda 0 split={split}")
