@@ -37,7 +37,7 @@ from attention_online_softmax_fwd_b200 import inputs as gen  # noqa: E402
 METRIC = "prefill attn TFLOPS & paged-decode KV-read GB/s, % of B200 roofline"
 PREFILL_CFG = "gqa_prefill_llama3_8b"
 DECODE_CFG = "paged_gqa_decode"
-DECODE_SPLIT = 1024
+DECODE_SPLIT = 256
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 

@@ -84,6 +84,10 @@ def test_long_context_decode_equals_prefill_last_row(cuda_device, workload):
 def dominant():
     q, k, v = gen.peaked_prefill_inputs(C["B"], C["Hq"], C["Hkv"], C["S"], C["D"], C["seed"] + 7, amp=12.0,
                                         period=C["S"])
+    # with ~99% of tiles dropped the output is close to V's row 0; V is scaled
+    # down so that the bf16 rounding of the output alone stays well inside the
+    # mean tolerance
+    v = (v.float() * 0.25).to(torch.bfloat16)
     cache = gen.paged_from_contiguous(q[:, C["S"] - 1], k, v, page_size=C["page_size"], seed=C["seed"] + 8)
     return q, k, v, cache
 
