@@ -133,6 +133,31 @@ def paged_from_contiguous(q_last, k, v, page_size, seed, poison=True):
                       torch.tensor([k.shape[1]], dtype=torch.int32), page_size)
 
 
+@dataclass
+class PagedPrefill:
+    q: torch.Tensor            # [B, Sq, Hq, D] bf16: queries of the Sq newest tokens
+    k_pages: torch.Tensor      # [P, page_size, Hkv, D] bf16, the new tokens' K/V included
+    v_pages: torch.Tensor
+    block_table: torch.Tensor  # [B, max_pages] int32
+    seq_lens: torch.Tensor     # [B] int32, total tokens per sequence (>= Sq)
+    k_seqs: list               # per sequence [L_b, Hkv, D] bf16 (contiguous copy)
+    v_seqs: list
+    page_size: int
+
+
+def paged_prefill_inputs(B, Sq, Hq, Hkv, D, page_size, lens, seed, poison=True, extra_frac=0.1):
+    """Chunked-prefill workload: each sequence b holds lens[b] >= Sq tokens of
+    K/V ~ N(0, 1) in a shared page pool (seeded permutation, NaN-poisoned spare
+    pages and tail slots); q ~ N(0, 1) for its Sq newest tokens."""
+    g = torch.Generator().manual_seed(seed)
+    q = _randn(g, (B, Sq, Hq, D)).to(torch.bfloat16)
+    k_seqs = [_randn(g, (int(L), Hkv, D)).to(torch.bfloat16) for L in lens]
+    v_seqs = [_randn(g, (int(L), Hkv, D)).to(torch.bfloat16) for L in lens]
+    k_pool, v_pool, bt = page_sequences(k_seqs, v_seqs, page_size, g, extra_frac, poison)
+    return PagedPrefill(q, k_pool, v_pool, bt, torch.tensor([int(L) for L in lens], dtype=torch.int32),
+                        k_seqs, v_seqs, page_size)
+
+
 # The workloads the library is measured and checked on (sizes as named).
 CONFIGS = {
     "tiny_gqa_prefill": dict(kind="prefill", B=1, Hq=4, Hkv=2, S=128, D=64, causal=True, seed=1001),

@@ -37,7 +37,11 @@ What it computes, and the passages it follows:
   of a unit in ascending key order; the result is the exact formula
   restricted to the kept keys.
 
-Parity status: dense prefill, paged decode and the gather are pinned by the
+* Chunked prefill over the paged cache (prefill_paged): the reading of
+  "chunked prefill" stated in its docstring.
+
+Parity status: dense prefill, paged decode, chunked paged prefill and the
+gather are pinned by the
 CPU tests (brute force, torch's float64 SDPA, closed forms, invariants). The
 BLASST walk is pinned against a brute-force recomputation of the rule from the
 full score matrix and against its invariants; the rule itself is a reading of
@@ -168,6 +172,47 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, page_size: int, sca
             kv = kv_head_of(hq, Hq, Hkv)
             ob, lb = attention_rows(q[b, hq][None, :], kb[:, kv, :], vb[:, kv, :], scale)
             o[b, hq], lse[b, hq] = ob[0], lb[0]
+    return o, lse
+
+
+def prefill_paged(q, k_pages, v_pages, block_table, seq_lens, page_size: int, scale: float,
+                  seqs=None, heads=None):
+    """Chunked (append) prefill over a paged KV cache.
+
+    The GQA page ("TensorRT对Grouped Query Attention的支持进展", section
+    与动态批处理协同) recommends chunked prefill and prefix caching for batches of
+    mixed lengths; the integration page ("flash-attention与TensorRT-LLM集成")
+    runs attention against a KV cache (flash_attn_with_kvcache). Neither spells
+    out the masking; the plainest reading, used here: the queries are the Sq
+    newest tokens of each sequence, whose keys and values are already in the
+    cache, and query row i of sequence b sits at position L_b - Sq + i and sees
+    the cached keys 0 .. L_b - Sq + i (causal, aligned at the end of the
+    sequence; L_b = seq_lens[b] >= Sq).
+
+    q [B, Sq, Hq, D]; k_pages/v_pages [P, page_size, Hkv, D]; block_table
+    [B, max_pages]; seq_lens [B]. Returns o [B, Sq, Hq, D] and lse [B, Hq, Sq]
+    (float64). ``seqs`` / ``heads`` (lists of b / hq) restrict the work to a
+    sample; entries outside it are NaN.
+    """
+    q = _f64(q)
+    bt = np.asarray(block_table)
+    lens = np.asarray(seq_lens)
+    B, Sq, Hq, D = q.shape
+    Hkv = k_pages.shape[2]
+    o = np.full((B, Sq, Hq, v_pages.shape[-1]), np.nan)
+    lse = np.full((B, Hq, Sq), np.nan)
+    for b in (range(B) if seqs is None else seqs):
+        L = int(lens[b])
+        if L < Sq:
+            raise ValueError(f"sequence {b}: {L} cached tokens for {Sq} queries")
+        kb = gather_pages(k_pages, bt[b], L, page_size)
+        vb = gather_pages(v_pages, bt[b], L, page_size)
+        vis = causal_visible(np.arange(Sq) + (L - Sq), L)
+        for hq in (range(Hq) if heads is None else heads):
+            kv = kv_head_of(hq, Hq, Hkv)
+            ob, lb = attention_rows(q[b, :, hq, :], kb[:, kv, :], vb[:, kv, :], scale, vis)
+            o[b, :, hq, :] = ob
+            lse[b, hq, :] = lb
     return o, lse
 
 

@@ -435,3 +435,83 @@ def test_blasst_decode_decisions_and_splits():
         grp = skip[0, kv] == 1
         for h in range(kv * G, kv * G + G):
             assert not (grp & ~(skip_h[0, h] == 1)).any()
+
+
+# ---------------------------------------------------------------- chunked prefill over pages
+
+def test_prefill_paged_matches_brute_force():
+    rng = np.random.default_rng(31)
+    B, Sq, Hq, Hkv, D, ps = 2, 3, 4, 2, 3, 4
+    lens = [5, 9]
+    P = 8
+    kp, vp = rng.standard_normal((P, ps, Hkv, D)), rng.standard_normal((P, ps, Hkv, D))
+    q = rng.standard_normal((B, Sq, Hq, D))
+    bt = np.array([[6, 1, -1], [0, 7, 3]])
+    o, lse = orc.prefill_paged(q, kp, vp, bt, lens, ps, 0.5)
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // 2
+            for i in range(Sq):
+                pos = lens[b] - Sq + i
+                ws = []
+                for j in range(pos + 1):
+                    page, slot = bt[b, j // ps], j % ps
+                    s_ = sum(q[b, i, h, d] * kp[page, slot, kv, d] for d in range(D)) * 0.5
+                    ws.append((page, slot, math.exp(s_)))
+                z = sum(e for *_, e in ws)
+                for d in range(D):
+                    ref = sum(e * vp[pg, sl, kv, d] for pg, sl, e in ws) / z
+                    assert abs(o[b, i, h, d] - ref) < 1e-12
+                assert abs(lse[b, h, i] - math.log(z)) < 1e-12
+
+
+def test_prefill_paged_whole_sequence_is_causal_prefill():
+    c = gen.paged_prefill_inputs(1, 50, 4, 2, 8, 16, [50], seed=32)
+    o, lse = orc.prefill_paged(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens, 16, 0.3)
+    op, lp = orc.prefill(c.q, c.k_seqs[0][None], c.v_seqs[0][None], True, 0.3)
+    np.testing.assert_allclose(o, op, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lp, rtol=0, atol=1e-13)
+
+
+def test_prefill_paged_single_query_is_decode():
+    c = gen.paged_prefill_inputs(3, 1, 8, 2, 8, 16, [1, 17, 60], seed=33)
+    o, lse = orc.prefill_paged(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens, 16, 0.4)
+    od, ld = orc.decode_paged(c.q[:, 0], c.k_pages, c.v_pages, c.block_table, c.seq_lens, 16, 0.4)
+    np.testing.assert_allclose(o[:, 0], od, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, :, 0], ld, rtol=0, atol=1e-13)
+
+
+def test_prefill_paged_chunks_compose():
+    # the last Sq1 + Sq2 tokens as one chunk equal two chunks: the first Sq1 of
+    # them against the cache up to their own end, then the last Sq2
+    c = gen.paged_prefill_inputs(2, 12, 4, 2, 8, 16, [40, 12], seed=34)
+    o, lse = orc.prefill_paged(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens, 16, 0.3)
+    Sq1 = 5
+    lens1 = c.seq_lens - (12 - Sq1)
+    o1, l1 = orc.prefill_paged(c.q[:, :Sq1], c.k_pages, c.v_pages, c.block_table, lens1, 16, 0.3)
+    o2, l2 = orc.prefill_paged(c.q[:, Sq1:], c.k_pages, c.v_pages, c.block_table, c.seq_lens, 16, 0.3)
+    np.testing.assert_allclose(o[:, :Sq1], o1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(o[:, Sq1:], o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, :, :Sq1], l1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, :, Sq1:], l2, rtol=0, atol=1e-13)
+
+
+def test_prefill_paged_matches_torch_sdpa_with_end_aligned_mask():
+    c = gen.paged_prefill_inputs(2, 9, 8, 2, 16, 16, [33, 9], seed=35, poison=False)
+    o, _ = orc.prefill_paged(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens, 16, 0.25)
+    for b in range(2):
+        L = int(c.seq_lens[b])
+        qb = c.q[b].double().permute(1, 0, 2)[None]                  # [1, Hq, Sq, D]
+        kb = c.k_seqs[b].double().permute(1, 0, 2)[None]             # [1, Hkv, L, D]
+        vb = c.v_seqs[b].double().permute(1, 0, 2)[None]
+        mask = torch.arange(L)[None, :] <= (torch.arange(9)[:, None] + (L - 9))
+        ref = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask, scale=0.25,
+                                                               enable_gqa=True)
+        np.testing.assert_allclose(o[b], ref[0].permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+
+
+def test_prefill_paged_rejects_short_cache():
+    c = gen.paged_prefill_inputs(1, 4, 2, 1, 8, 16, [4], seed=36)
+    with pytest.raises(ValueError):
+        orc.prefill_paged(c.q, c.k_pages, c.v_pages, c.block_table, torch.tensor([3]), 16, 0.3)
+
