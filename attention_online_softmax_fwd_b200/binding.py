@@ -45,6 +45,7 @@ SIGNATURES = {
     "attn_abi_version": (_I, []),
     "attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "attn_prefill_blasst": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P]),
+    "attn_prefill_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
     "attn_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                _P, _SZ, _P, _P, _P]),
@@ -134,6 +135,29 @@ def prefill(q, k, v, causal: bool = True, scale: float | None = None, out=None, 
     st = load_library().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, S, D,
                                      int(bool(causal)), scale, _stream_handle(stream))
     _check(st, "attn_prefill")
+    return o, lse
+
+
+def prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float | None = None, out=None, lse=None,
+                  device_status=None, return_lse: bool = True, stream=None):
+    """Chunked prefill over a paged KV cache: q [B,Sq,Hq,D] bf16 are the Sq newest
+    tokens of each sequence (their K/V already in the pages); row i of sequence b
+    sees its cached keys 0 .. seq_lens[b] - Sq + i. -> (o [B,Sq,Hq,D], lse [B,Hq,Sq])."""
+    _need(q, torch.bfloat16, 4, "q")
+    _need(k_pages, torch.bfloat16, 4, "k_pages")
+    _need(v_pages, torch.bfloat16, 4, "v_pages")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    B, Sq, Hq, D = q.shape
+    P, page_size, Hkv, _ = k_pages.shape
+    scale = default_scale(D) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_prefill_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), _ptr(o), _ptr(lse), B, Sq, Hq,
+        Hkv, D, page_size, block_table.shape[1], P, scale, _ptr(device_status), _stream_handle(stream))
+    _check(st, "attn_prefill_paged")
     return o, lse
 
 

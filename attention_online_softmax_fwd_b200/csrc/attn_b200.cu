@@ -104,10 +104,10 @@ int encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int D) 
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
 
-template <int D, bool CAUSAL, bool SKIP>
+template <int D, bool CAUSAL, bool SKIP, bool PAGED = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
                    int sms, cudaStream_t stream) {
-  auto kernel = prefill_kernel<D, CAUSAL, SKIP>;
+  auto kernel = prefill_kernel<D, CAUSAL, SKIP, PAGED>;
   constexpr int smem = PrefillSmem<D>::kDynamic;
   // The kernel moves registers between warpgroups with setmaxnreg; the block's
   // launch allocation must cover the split or the increase would never return.
@@ -168,6 +168,17 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   return use_skip ? dispatch_prefill_causal<64, true>(causal != 0, tq, tk, tv, p, sms, s)
                   : dispatch_prefill_causal<64, false>(causal != 0, tq, tk, tv, p, sms, s);
 }
+
+// Page pool [P][page_size][Hkv][D] as a 4-D map {D, Hkv, page_size, P}; box =
+// 64 columns x 16 slots of one head (a page size is a multiple of 16).
+int encode_pool16(CUtensorMap* map, const void* base, int P, int page_size, int Hkv, int D) {
+  const uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(page_size), uint64_t(P)};
+  const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(Hkv) * D * 2, uint64_t(page_size) * Hkv * D * 2};
+  const uint32_t box[4] = {64, 1, 16, 1};
+  return encode_map(map, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool valid_prefill_page_size(int ps) { return ps == 16 || ps == 32 || ps == 64 || ps == 128 || ps == 256; }
 
 // ------------------------------------------------------------------ decode
 
@@ -277,6 +288,53 @@ int attn_prefill_blasst(const void* q, const void* k, const void* v, void* o, fl
                         int* device_status, void* stream) {
   return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, lambda, skip_mask, device_status, stream,
                       true);
+}
+
+int attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                       const int32_t* seq_lens, void* o, float* lse, int B, int Sq, int Hq, int Hkv, int D,
+                       int page_size, int max_pages_per_seq, int num_pages, float scale, int* device_status,
+                       void* stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Sq < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!valid_prefill_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+  if ((long long)Sq > (long long)max_pages_per_seq * page_size) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Sq * Hq > (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  int sms = 0;
+  if (int st = current_device(&sms)) return st;
+
+  PrefillParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.status = device_status;
+  p.B = B; p.S = Sq; p.Hq = Hq; p.Hkv = Hkv;
+  p.n_qblocks = (Sq + 2 * kPfRows - 1) / (2 * kPfRows);
+  p.n_qt = (Sq + kPfRows - 1) / kPfRows;
+  p.n_kt = 0;
+  const long long num_items = (long long)p.n_qblocks * B * Hq;
+  if (num_items > 0x7fffffffll) return ATTN_ERR_UNSUPPORTED;
+  p.num_items = int(num_items);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.log2_lambda = -INFINITY;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.k_pool = static_cast<const __nv_bfloat16*>(k_pages);
+  p.v_pool = static_cast<const __nv_bfloat16*>(v_pages);
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+
+  CUtensorMap tq, tk, tv;
+  if (int st = encode_bshd(&tq, q, B, Sq, Hq, D)) return st;
+  if (int st = encode_pool16(&tk, k_pages, num_pages, page_size, Hkv, D)) return st;
+  if (int st = encode_pool16(&tv, v_pages, num_pages, page_size, Hkv, D)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_prefill<128, true, false, true>(tq, tk, tv, p, sms, s)
+                  : launch_prefill<64, true, false, true>(tq, tk, tv, p, sms, s);
 }
 
 size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq, int page_size,

@@ -42,6 +42,12 @@ struct PrefillParams {
   int num_items;       // n_qblocks * B * Hq (< 2^31)
   float scale_log2;    // scale * log2(e)
   float log2_lambda;   // log2(lambda) (tile skip only)
+  // chunked prefill over a paged cache (S is then the chunk length Sq)
+  const int* block_table;  // [B][max_pages]
+  const int* seq_lens;     // [B]: tokens in the cache, the chunk's own included (>= S)
+  const __nv_bfloat16* k_pool;   // [num_pages][page_size][Hkv][D]
+  const __nv_bfloat16* v_pool;
+  int max_pages, num_pages, page_size;
 };
 
 constexpr int kPfRows = 128;     // rows per query tile
@@ -196,6 +202,55 @@ __device__ __forceinline__ void pf_load_scores(uint32_t taddr, float (&s)[kPfKey
   }
 }
 
+// Zero source for the paged loads of key slots past a sequence's end.
+__device__ __align__(16) uint8_t g_pf_zero16[16];
+
+// One K or V tile of 128 keys gathered from the page pool (chunked prefill):
+// 16 keys per copy (page sizes are multiples of 16, so a group never straddles
+// two pages), completing on `bar` for kTileBytes in all. A group wholly past
+// the sequence end, or in a page the block table does not hold (reported as
+// ATTN_ERR_DEVICE_BOUNDS), is filled with zeros by an out-of-range page
+// coordinate, which reads nothing. The group holding the sequence end is
+// copied 16 bytes at a time into the swizzled positions, zeros past the end,
+// so no slot past the end is read: those slots may hold anything, and a NaN
+// there would survive a zero probability in P V.
+template <int D>
+__device__ __forceinline__ void pf_load_paged_tile(uint8_t* dst, const CUtensorMap* tm16, const __nv_bfloat16* pool,
+                                                   uint64_t* bar, const PrefillParams& p, int b, int kvh, int key0,
+                                                   int n_keys) {
+  const int* bt = p.block_table + size_t(b) * p.max_pages;
+#pragma unroll 1
+  for (int g = 0; g < kPfKeys / 16; ++g) {
+    const int key = key0 + g * 16;
+    const int lp = key / p.page_size;
+    const int slot0 = key % p.page_size;
+    int phys = p.num_pages;   // out of range: zeros
+    if (key < n_keys && lp < p.max_pages) {
+      const int e = __ldg(&bt[lp]);
+      if (e >= 0 && e < p.num_pages) phys = e;
+      else raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
+    }
+    if (key + 16 <= n_keys || phys == p.num_pages) {
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_4d(dst + c * (kPfRows * 128) + g * 16 * 128, tm16, bar, c * 64, kvh, slot0, phys);
+    } else {
+      for (int r = 0; r < 16; ++r) {
+        const int row = g * 16 + r;
+        const bool valid = key + r < n_keys;
+        const uint8_t* src_row = reinterpret_cast<const uint8_t*>(
+            pool + ((size_t(phys) * p.page_size + slot0 + r) * p.Hkv + kvh) * D);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            bulk_load(dst + c * (kPfRows * 128) + row * 128 + ((u ^ (row & 7)) << 4),
+                      valid ? src_row + c * 128 + u * 16 : g_pf_zero16, 16, bar);
+      }
+    }
+  }
+}
+
 // Record the decisions for K/V tile jt (two 64-key tiles) of query tile qt:
 // 1 skipped, 0 kept; tiles past the causal diagonal or the sequence stay untouched.
 template <bool CAUSAL>
@@ -210,7 +265,12 @@ __device__ __forceinline__ void pf_write_skip_mask(const PrefillParams& p, int b
   }
 }
 
-template <int D, bool CAUSAL, bool SKIP>
+// PAGED: chunked prefill. Query row i of sequence b sits at position
+// L_b - S + i (L_b = seq_lens[b]) and sees cached keys 0 .. L_b - S + i; the K
+// and V tiles are gathered from the page pool through the block table, one
+// box of 16 keys at a time (pf_load_paged_tile; tm_k / tm_v then map the pools as
+// {D, Hkv, page_size, P} with 16-slot boxes).
+template <int D, bool CAUSAL, bool SKIP, bool PAGED = false>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -267,9 +327,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     hq = rem % p.Hq;
   };
   auto tile_rows = [&](int qb, int x) { return max(0, min(kPfRows, p.S - qb * 2 * kPfRows - x * kPfRows)); };
-  auto tile_nkv = [&](int qb, int x, int rows) {
+  // PAGED: position of query row 0 of sequence b (its cache length minus the
+  // chunk length); a length outside [S, capacity] is clamped and, when asked,
+  // reported as ATTN_ERR_DEVICE_BOUNDS
+  auto seq_offset = [&](int b, bool report) {
+    if constexpr (!PAGED) {
+      return 0;
+    } else {
+      const int cap = p.max_pages * p.page_size;
+      int len = __ldg(&p.seq_lens[b]);
+      if (len < p.S || len > cap) {
+        if (report) raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
+        len = max(p.S, min(len, cap));
+      }
+      return len - p.S;
+    }
+  };
+  auto tile_nkv = [&](int qb, int x, int rows, int off) {
     if (rows == 0) return 0;
-    if (CAUSAL) return (qb * 2 * kPfRows + x * kPfRows + rows - 1) / kPfKeys + 1;
+    if (CAUSAL) return (off + qb * 2 * kPfRows + x * kPfRows + rows - 1) / kPfKeys + 1;
     return (p.S + kPfKeys - 1) / kPfKeys;
   };
 
@@ -292,8 +368,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           int qb, b, hq;
           item_coords(item, qb, b, hq);
           const int kvh = hq / (p.Hq / p.Hkv);
+          const int off = seq_offset(b, false);
           const int rows0 = tile_rows(qb, 0), rows1 = tile_rows(qb, 1);
-          const int n = max(tile_nkv(qb, 0, rows0), tile_nkv(qb, 1, rows1));
+          const int n = max(tile_nkv(qb, 0, rows0, off), tile_nkv(qb, 1, rows1, off));
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if ((x == 0 ? rows0 : rows1) == 0 || !ok) continue;
@@ -314,10 +391,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
             mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
             const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+            if constexpr (PAGED) {
+              pf_load_paged_tile<D>(smem + L::kRing + slot * L::kTileBytes, tm, is_k ? p.k_pool : p.v_pool,
+                                    &bars[L::bKVFull + slot], p, b, kvh, key0, off + p.S);
+            } else {
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_4d(smem + L::kRing + slot * L::kTileBytes + c * L::kChunkBytes, tm, &bars[L::bKVFull + slot],
-                          c * 64, key0, kvh, b);
+              for (int c = 0; c < D / 64; ++c)
+                tma_load_4d(smem + L::kRing + slot * L::kTileBytes + c * L::kChunkBytes, tm,
+                            &bars[L::bKVFull + slot], c * 64, key0, kvh, b);
+            }
             pend_mask |= 1u << slot;
             pend_ph = (pend_ph & ~(1u << slot)) | (phase << slot);
             if (++slot == NS) { slot = 0; phase ^= 1u; }
@@ -350,9 +432,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
           int qb, b, hq;
           item_coords(item, qb, b, hq);
+          const int off = seq_offset(b, false);
           const int rows0 = tile_rows(qb, 0), rows1 = tile_rows(qb, 1);
-          const int n = max(tile_nkv(qb, 0, rows0), tile_nkv(qb, 1, rows1));
-          const int nkv = tile_nkv(qb, x, x == 0 ? rows0 : rows1);
+          const int n = max(tile_nkv(qb, 0, rows0, off), tile_nkv(qb, 1, rows1, off));
+          const int nkv = tile_nkv(qb, x, x == 0 ? rows0 : rows1, off);
           if (nkv > 0) {
             if (!mbar_wait(&bars[L::bQFull + x], qf_ph, abort_flag, p.status)) break;
             qf_ph ^= 1u;
@@ -435,8 +518,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
       int qb, b, hq;
       item_coords(item, qb, b, hq);
+      const int off = seq_offset(b, x == 0 && t == 0);
+      const int n_keys = PAGED ? off + p.S : p.S;   // keys in the cache (the sequence)
       const int rows = tile_rows(qb, x);
-      const int nkv = tile_nkv(qb, x, rows);
+      const int nkv = tile_nkv(qb, x, rows, off);
       if (nkv == 0) continue;
       const int row0 = qb * 2 * kPfRows + x * kPfRows;
       const int row = row0 + t;
@@ -455,7 +540,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         const int key0 = j * kPfKeys;
         float s[kPfKeys];
-        pf_load_scores<CAUSAL>(taddr_s, s, key0, row, row0, p.S);
+        pf_load_scores<CAUSAL>(taddr_s, s, key0, off + row, off + row0, n_keys);
         if constexpr (!SKIP) {
           // S_x is in registers: the tensor pipe may overwrite it with the next tile
           tc_fence_before();
@@ -512,7 +597,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             decision = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status);
             if (decision < 0) { ok = false; break; }
             skip_all = decision == 3;
-            if (!skip_all) pf_load_scores<CAUSAL>(taddr_s, s, key0, row, row0, p.S);
+            if (!skip_all) pf_load_scores<CAUSAL>(taddr_s, s, key0, off + row, off + row0, n_keys);
           }
           tc_fence_before();
           __syncwarp();

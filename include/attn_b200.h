@@ -103,6 +103,36 @@ int attn_prefill_blasst(const void* q, const void* k, const void* v, void* o, fl
                         void* stream);
 
 /*
+ * attn_prefill_paged -- chunked (append) prefill over a paged KV cache
+ * ("TensorRT对Grouped Query Attention的支持进展", section 与动态批处理协同,
+ * recommends chunked prefill and prefix caching; "flash-attention与TensorRT-LLM
+ * 集成" runs attention against a KV cache). Causal, aligned at the end of each
+ * sequence: query row i of sequence b is the token at position L_b - Sq + i
+ * (L_b = seq_lens[b]) and sees the cached keys 0 .. L_b - Sq + i. The chunk's
+ * own keys and values must already be in the pages.
+ *
+ *   q            [B][Sq][Hq][D] bf16          the chunk's queries
+ *   k_pages,
+ *   v_pages      [num_pages][page_size][Hkv][D] bf16   the page pool
+ *   block_table  [B][max_pages_per_seq] int32 (device)
+ *   seq_lens     [B] int32 (device)   L_b, with Sq <= L_b <= max_pages_per_seq * page_size;
+ *                a length outside is clamped into that range and ATTN_ERR_DEVICE_BOUNDS set
+ *   o            [B][Sq][Hq][D] bf16 (out)
+ *   lse          [B][Hq][Sq] fp32 natural-log LSE (out), may be NULL
+ *   page_size    16, 32, 64, 128 or 256;  D 64 or 128;  Hq a multiple of Hkv
+ *   device_status  may be NULL (see attn_prefill_blasst)
+ * A block_table entry outside [0, num_pages) for a page the sequence uses is
+ * never dereferenced: its keys read as zeros and ATTN_ERR_DEVICE_BOUNDS is set.
+ * Cache slots past L_b are never read. Pointers: the bf16 ones 16-byte aligned.
+ * Errors as attn_prefill.
+ */
+int attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
+                       const int32_t* block_table, const int32_t* seq_lens, void* o, float* lse,
+                       int B, int Sq, int Hq, int Hkv, int D, int page_size,
+                       int max_pages_per_seq, int num_pages, float scale,
+                       int* device_status, void* stream);
+
+/*
  * attn_decode_workspace_bytes -- scratch needed by attn_decode_paged.
  * The decode splits each sequence's keys into chunks of split_tokens tokens,
  * computes one partial (O, LSE) per (sequence, query head, chunk), and merges

@@ -122,3 +122,24 @@ def test_binding_fails_loudly_when_library_missing(monkeypatch):
     monkeypatch.setattr(binding, "lib_path", lambda: "/nonexistent/libattn_b200.so")
     with pytest.raises(binding.AttnError):
         binding.load_library()
+
+
+def _paged_prefill(lib, **kw):
+    a = dict(q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=None, B=2, Sq=64, Hq=8, Hkv=2, D=128,
+             ps=16, mp=16, P=64, scale=0.09)
+    a.update(kw)
+    return lib.attn_prefill_paged(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["o"], a["lse"], a["B"], a["Sq"],
+                                  a["Hq"], a["Hkv"], a["D"], a["ps"], a["mp"], a["P"], a["scale"], None, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(bt=None), dict(sl=None), dict(o=None),
+                                 dict(kp=ctypes.c_void_p((1 << 20) + 8)), dict(bt=ctypes.c_void_p((1 << 20) + 2)),
+                                 dict(B=0), dict(Sq=0), dict(Hq=6, Hkv=4), dict(ps=24), dict(ps=8), dict(ps=512),
+                                 dict(mp=0), dict(P=0), dict(Sq=257, mp=16, ps=16), dict(scale=0.0),
+                                 dict(scale=float("inf"))])
+def test_prefill_paged_rejects_bad_arguments(lib, bad):
+    assert _paged_prefill(lib, **bad) == INVALID
+
+
+def test_prefill_paged_rejects_unsupported_head_dim(lib):
+    assert _paged_prefill(lib, D=96) == UNSUPPORTED
