@@ -205,48 +205,52 @@ __device__ __forceinline__ void pf_load_scores(uint32_t taddr, float (&s)[kPfKey
 // Zero source for the paged loads of key slots past a sequence's end.
 __device__ __align__(16) uint8_t g_pf_zero16[16];
 
-// One K or V tile of 128 keys gathered from the page pool (chunked prefill):
-// 16 keys per copy (page sizes are multiples of 16, so a group never straddles
-// two pages), completing on `bar` for kTileBytes in all. A group wholly past
+// Group g (16 keys) of a K or V tile of 128 keys gathered from the page pool
+// (chunked prefill): page sizes are multiples of 16, so a group never
+// straddles two pages; the eight groups of a tile complete on `bar` for
+// kTileBytes in all. A group wholly past
 // the sequence end, or in a page the block table does not hold (reported as
 // ATTN_ERR_DEVICE_BOUNDS), is filled with zeros by an out-of-range page
 // coordinate, which reads nothing. The group holding the sequence end is
 // copied 16 bytes at a time into the swizzled positions, zeros past the end,
 // so no slot past the end is read: those slots may hold anything, and a NaN
 // there would survive a zero probability in P V.
+// The raw block-table entry of group g of K/V tile t of sequence b, or
+// num_pages (nothing to read) for a group past the sequence end.
+__device__ __forceinline__ int pf_page_entry(const PrefillParams& p, int b, int t, int g, int n_keys) {
+  const int key = t * kPfKeys + g * 16;
+  const int lp = key / p.page_size;
+  return (key < n_keys && lp < p.max_pages) ? __ldg(&p.block_table[size_t(b) * p.max_pages + lp]) : p.num_pages;
+}
+
 template <int D>
-__device__ __forceinline__ void pf_load_paged_tile(uint8_t* dst, const CUtensorMap* tm16, const __nv_bfloat16* pool,
-                                                   uint64_t* bar, const PrefillParams& p, int b, int kvh, int key0,
-                                                   int n_keys) {
-  const int* bt = p.block_table + size_t(b) * p.max_pages;
-#pragma unroll 1
-  for (int g = 0; g < kPfKeys / 16; ++g) {
-    const int key = key0 + g * 16;
-    const int lp = key / p.page_size;
-    const int slot0 = key % p.page_size;
-    int phys = p.num_pages;   // out of range: zeros
-    if (key < n_keys && lp < p.max_pages) {
-      const int e = __ldg(&bt[lp]);
-      if (e >= 0 && e < p.num_pages) phys = e;
-      else raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
-    }
-    if (key + 16 <= n_keys || phys == p.num_pages) {
+__device__ __forceinline__ void pf_load_paged_group(uint8_t* dst, const CUtensorMap* tm16,
+                                                    const __nv_bfloat16* pool, uint64_t* bar,
+                                                    const PrefillParams& p, int kvh, int key0, int n_keys, int g,
+                                                    int entry) {
+  const int key = key0 + g * 16;
+  const int slot0 = key % p.page_size;
+  int phys = p.num_pages;   // out of range: zeros
+  if (key < n_keys) {
+    if (entry >= 0 && entry < p.num_pages) phys = entry;
+    else raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
+  }
+  if (key + 16 <= n_keys || phys == p.num_pages) {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c)
+      tma_load_4d(dst + c * (kPfRows * 128) + g * 16 * 128, tm16, bar, c * 64, kvh, slot0, phys);
+  } else {
+    for (int r = 0; r < 16; ++r) {
+      const int row = g * 16 + r;
+      const bool valid = key + r < n_keys;
+      const uint8_t* src_row =
+          reinterpret_cast<const uint8_t*>(pool + ((size_t(phys) * p.page_size + slot0 + r) * p.Hkv + kvh) * D);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
-        tma_load_4d(dst + c * (kPfRows * 128) + g * 16 * 128, tm16, bar, c * 64, kvh, slot0, phys);
-    } else {
-      for (int r = 0; r < 16; ++r) {
-        const int row = g * 16 + r;
-        const bool valid = key + r < n_keys;
-        const uint8_t* src_row = reinterpret_cast<const uint8_t*>(
-            pool + ((size_t(phys) * p.page_size + slot0 + r) * p.Hkv + kvh) * D);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            bulk_load(dst + c * (kPfRows * 128) + row * 128 + ((u ^ (row & 7)) << 4),
-                      valid ? src_row + c * 128 + u * 16 : g_pf_zero16, 16, bar);
-      }
+        for (int u = 0; u < 8; ++u)
+          bulk_load(dst + c * (kPfRows * 128) + row * 128 + ((u ^ (row & 7)) << 4),
+                    valid ? src_row + c * 128 + u * 16 : g_pf_zero16, 16, bar);
     }
   }
 }
@@ -353,7 +357,78 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   // (kPfRegPoolNeeded is checked against the launch allocation on the host).
   if (warp < 4) {
     setmaxnreg_dec<kPfRegsLow>();
-    if (warp == kPfProducerWarp) {
+    if (warp == kPfProducerWarp && PAGED) {
+      // ============================================================ TMA producer (paged)
+      // Lane 0 waits for free slots and arms the barriers; lanes 0-7 each copy
+      // one 16-key group of a tile, so the block-table loads and the copies of a
+      // tile are issued in parallel.
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+      }
+      int slot = 0;
+      uint32_t phase = 0;
+      uint32_t qe_bits = 3u;
+      uint32_t pend_mask = 0, pend_ph = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+        int qb, b, hq;
+        item_coords(item, qb, b, hq);
+        const int kvh = hq / (p.Hq / p.Hkv);
+        const int off = seq_offset(b, false);
+        const int rows0 = tile_rows(qb, 0), rows1 = tile_rows(qb, 1);
+        const int n = max(tile_nkv(qb, 0, rows0, off), tile_nkv(qb, 1, rows1, off));
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if ((x == 0 ? rows0 : rows1) == 0 || !ok) continue;
+          int w = 1;
+          if (lane == 0) w = mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; continue; }
+          qe_bits ^= 1u << x;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bars[L::bQFull + x], L::kTileBytes);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_4d(smem + L::kQ + x * L::kTileBytes + c * L::kChunkBytes, &tm_q, &bars[L::bQFull + x],
+                          c * 64, qb * 2 * kPfRows + x * kPfRows, hq, b);
+          }
+        }
+        // Block-table entries: this lane's group of the next K tile is fetched
+        // one K tile ahead; V_t reuses the entry of K_t.
+        const int n_keys = off + p.S;
+        const int g = lane & 7;
+        int pre = pf_page_entry(p, b, 0, g, n_keys);
+        int entry_even = p.num_pages, entry_odd = p.num_pages;   // of the last K tiles with even / odd index
+        for (int step = 0; step < 2 * n && ok; ++step) {
+          const int j = (step - 1) / 2;
+          const bool is_k = step == 0 || (step % 2 == 1 && j + 1 < n);
+          const int key0 = step == 0 ? 0 : (is_k ? (j + 1) * kPfKeys : (step % 2 == 1 ? j : step / 2 - 1) * kPfKeys);
+          const int tile = key0 / kPfKeys;
+          if (is_k) {
+            if (tile & 1) entry_odd = pre; else entry_even = pre;
+            pre = pf_page_entry(p, b, tile + 1, g, n_keys);
+          }
+          const int entry = (tile & 1) ? entry_odd : entry_even;
+          int w = 1;
+          if (lane == 0) w = mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+          if (lane == 0) mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
+          if (lane < kPfKeys / 16)
+            pf_load_paged_group<D>(smem + L::kRing + slot * L::kTileBytes, is_k ? &tm_k : &tm_v,
+                                   is_k ? p.k_pool : p.v_pool, &bars[L::bKVFull + slot], p, kvh, key0, n_keys,
+                                   lane, entry);
+          pend_mask |= 1u << slot;
+          pend_ph = (pend_ph & ~(1u << slot)) | (phase << slot);
+          if (++slot == NS) { slot = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && lane == 0) {
+        for (int s = 0; s < NS; ++s)
+          if (pend_mask & (1u << s)) mbar_drain(&bars[L::bKVFull + s], (pend_ph >> s) & 1u);
+      }
+      __syncwarp();
+    } else if (warp == kPfProducerWarp) {
       // ============================================================ TMA producer
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
@@ -391,15 +466,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
             mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
             const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
-            if constexpr (PAGED) {
-              pf_load_paged_tile<D>(smem + L::kRing + slot * L::kTileBytes, tm, is_k ? p.k_pool : p.v_pool,
-                                    &bars[L::bKVFull + slot], p, b, kvh, key0, off + p.S);
-            } else {
 #pragma unroll
-              for (int c = 0; c < D / 64; ++c)
-                tma_load_4d(smem + L::kRing + slot * L::kTileBytes + c * L::kChunkBytes, tm,
-                            &bars[L::bKVFull + slot], c * 64, key0, kvh, b);
-            }
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_4d(smem + L::kRing + slot * L::kTileBytes + c * L::kChunkBytes, tm, &bars[L::bKVFull + slot],
+                          c * 64, key0, kvh, b);
             pend_mask |= 1u << slot;
             pend_ph = (pend_ph & ~(1u << slot)) | (phase << slot);
             if (++slot == NS) { slot = 0; phase ^= 1u; }

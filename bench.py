@@ -366,12 +366,42 @@ def run_gpu(args, world, rank, local):
     }
     if rank == 0 and world == 1 and not args.no_blasst:
         line["blasst_long_context"] = blasst_long_context_report(dev)
+        line["chunked_prefill_paged"] = chunked_prefill_report(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfs, gbs, secs, desc = oracle_sample(int(args.cpu_heads), 4)
         line["cpu_baseline"] = {"value": tfs, "unit": "TFLOP/s", "cores": cpu_threads()[0], "kind": "oracle",
                                 "sample": desc, "decode_gbs": gbs, "seconds": secs}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def chunked_prefill_report(dev, peaks, reps=5):
+    """Chunked prefill over the paged cache: 4 sequences, 2048 new tokens each
+    after cached prefixes of 0, 2048, 4096 and 6144 tokens (Hq 32, Hkv 8, D 128,
+    16-token pages). FLOPs: 4 D per visible (query, key) pair."""
+    import attention_online_softmax_fwd_b200 as ab
+    B, Sq, Hq, Hkv, D, ps = 4, 2048, 32, 8, 128, 16
+    lens = [2048, 4096, 6144, 8192]
+    c = gen.paged_prefill_inputs(B, Sq, Hq, Hkv, D, ps, lens, seed=1006)
+    args = [t.to(dev) for t in (c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens)]
+    scale = gen.attn_scale(D)
+    pairs = sum(Sq * (L - Sq) + Sq * (Sq + 1) // 2 for L in lens)
+    fl = 4.0 * D * Hq * pairs
+    stream = torch.cuda.current_stream(dev)
+    ab.prefill_paged(*args, scale=scale)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ab.prefill_paged(*args, scale=scale)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.median(ts)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": "B4 Sq2048 after prefixes 0/2048/4096/6144, Hq32 Hkv8 D128, 16-token pages",
+            "ms": ms, "tflops": tf, "flops": fl, "frac_of_measured_bf16": tf / peaks["bf16_tflops"]}
 
 
 def blasst_long_context_report(dev, reps=3):
