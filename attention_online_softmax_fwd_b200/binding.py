@@ -49,6 +49,8 @@ SIGNATURES = {
     "attn_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                _P, _SZ, _P, _P, _P]),
+    "attn_decode_paged_blasst_heads": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P,
+                                            _P, _P, _SZ, _P, _P, _P]),
     "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                        _P, _P, _P]),
     "attn_read_device_status": (_I, [ctypes.POINTER(_I), _I]),
@@ -195,7 +197,7 @@ def decode_skip_mask_shape(num_seqs, Hkv, max_pages, page_size):
 
 
 def _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens, out, lse, workspace,
-            skip_mask, device_status, return_lse, stream):
+            skip_mask, device_status, return_lse, stream, per_head=False):
     _need(q, torch.bfloat16, 3, "q")
     _need(k_pages, torch.bfloat16, 4, "k_pages")
     _need(v_pages, torch.bfloat16, 4, "v_pages")
@@ -217,15 +219,16 @@ def _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     mask = None
     if skip_mask is True:
-        mask = torch.full(decode_skip_mask_shape(N, Hkv, max_pages, page_size), 2, dtype=torch.uint8,
-                          device=q.device)
+        mask = torch.full(decode_skip_mask_shape(N, Hq if per_head else Hkv, max_pages, page_size), 2,
+                          dtype=torch.uint8, device=q.device)
     elif isinstance(skip_mask, torch.Tensor):
         mask = skip_mask
-    st = load_library().attn_decode_paged(
+    fn = load_library().attn_decode_paged_blasst_heads if per_head else load_library().attn_decode_paged
+    st = fn(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), N, Hq, Hkv, D, page_size,
         max_pages, P, scale, lam, split_tokens, _ptr(o), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(mask), _ptr(device_status), _stream_handle(stream))
-    _check(st, "attn_decode_paged")
+    _check(st, "attn_decode_paged_blasst_heads" if per_head else "attn_decode_paged")
     return o, lse, mask
 
 
@@ -239,10 +242,16 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, split_t
 
 def decode_paged_blasst(q, k_pages, v_pages, block_table, seq_lens, lam: float, scale=None,
                         split_tokens: int = 1024, out=None, lse=None, workspace=None, skip_mask=True,
-                        device_status=None, return_lse=True, stream=None):
-    """Paged decode with the BLASST tile skip. Returns (o, lse, skip_mask)."""
+                        device_status=None, return_lse=True, stream=None, rows_per_unit: str = "group"):
+    """Paged decode with the BLASST tile skip. Returns (o, lse, skip_mask).
+
+    rows_per_unit="group": one decision per (sequence, KV head, tile) for the G
+    query heads that share the KV head (mask [N, Hkv, tiles]); "head": one per
+    query head (mask [N, Hq, tiles])."""
+    if rows_per_unit not in ("group", "head"):
+        raise AttnError("rows_per_unit must be 'group' or 'head'")
     return _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens, out, lse,
-                   workspace, skip_mask, device_status, return_lse, stream)
+                   workspace, skip_mask, device_status, return_lse, stream, per_head=rows_per_unit == "head")
 
 
 def decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale=None, split_tokens: int = 1024,

@@ -348,11 +348,11 @@ size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_pe
   return kWsHeader + o_bytes_aligned + size_t(num_seqs) * ms * Hq * sizeof(float);
 }
 
-int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
-                      const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
-                      int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens, void* o,
-                      float* lse, void* workspace, size_t workspace_bytes, uint8_t* skip_mask, int* device_status,
-                      void* stream) {
+static int decode_impl(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                       const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
+                       int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens, void* o,
+                       float* lse, void* workspace, size_t workspace_bytes, uint8_t* skip_mask,
+                       int* device_status, void* stream, bool per_head) {
   if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace))
     return ATTN_ERR_INVALID_ARG;
@@ -391,6 +391,7 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   p.chunk = page_size < 64 ? page_size : 64;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.log2_lambda = lambda > 0.f ? std::log2(lambda) : -INFINITY;
+  p.per_head = per_head ? 1 : 0;
   p.num_items = (long long)num_seqs * ms * Hkv;
 
   // page pool [P][page_size][Hkv][D] as a 5-D map {64, D/64, Hkv, page_size, P}; box = the whole head
@@ -402,7 +403,7 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   if (int st = encode_map5(&tk, k_pages, dims, strides, box)) return st;
   if (int st = encode_map5(&tv, v_pages, dims, strides, box)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool use_skip = lambda > 0.f || skip_mask != nullptr;
+  const bool use_skip = lambda > 0.f || skip_mask != nullptr || per_head;
   const int hg = Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0);
   if (!use_skip && hg > 0) {
     // dense: one item per group of hg KV heads, 16-token stages covering all of them
@@ -421,6 +422,26 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
                     : dispatch_decode_g<128, false>(G, tk, tv, p, sms, s);
   return use_skip ? dispatch_decode_g<64, true>(G, tk, tv, p, sms, s)
                   : dispatch_decode_g<64, false>(G, tk, tv, p, sms, s);
+}
+
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                      const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
+                      int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens, void* o,
+                      float* lse, void* workspace, size_t workspace_bytes, uint8_t* skip_mask, int* device_status,
+                      void* stream) {
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, num_seqs, Hq, Hkv, D, page_size,
+                     max_pages_per_seq, num_pages, scale, lambda, split_tokens, o, lse, workspace, workspace_bytes,
+                     skip_mask, device_status, stream, false);
+}
+
+int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const void* v_pages,
+                                   const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int Hq,
+                                   int Hkv, int D, int page_size, int max_pages_per_seq, int num_pages, float scale,
+                                   float lambda, int split_tokens, void* o, float* lse, void* workspace,
+                                   size_t workspace_bytes, uint8_t* skip_mask, int* device_status, void* stream) {
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, num_seqs, Hq, Hkv, D, page_size,
+                     max_pages_per_seq, num_pages, scale, lambda, split_tokens, o, lse, workspace, workspace_bytes,
+                     skip_mask, device_status, stream, true);
 }
 
 }  // extern "C"

@@ -38,13 +38,14 @@ struct DecodeParams {
   float* lse;                  // [N][Hq] (natural log) or null
   float* ws_o;                 // [N][max_splits][Hq][D] fp32 partial outputs (normalised)
   float* ws_lse;               // [N][max_splits][Hq] fp32 partial log2-sum-exp
-  uint8_t* skip_mask;          // [N][Hkv][max_tiles] or null
+  uint8_t* skip_mask;          // [N][Hkv][max_tiles] (per_head: [N][Hq][max_tiles]) or null
   int* status;                 // caller's device status word or null
   int num_seqs, Hq, Hkv, page_size, max_pages, num_pages;
   int split_tokens, max_splits, max_tiles;
   int chunk;          // tokens per TMA copy: min(page_size, 64)
   float scale_log2;   // softmax scale * log2(e)
   float log2_lambda;  // log2(lambda) for the tile skip
+  int per_head;       // tile skip decided for each query head alone, not for the KV head's group
   long long num_items;
 };
 
@@ -367,6 +368,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
 
       bool skip = false;
+      bool skip_r[2] = {false, false};   // per_head: this lane's rows g, g + 8 drop the tile
       if constexpr (SKIP) {
         // tile row maxima over all four warps, then the unit-wide decision
         if (tq == 0) {
@@ -388,14 +390,34 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           const bool ok_r = !valid_row || r[rr] == neg_inf ||
                             (m_true[rr] != neg_inf && (r[rr] - m_true[rr]) < p.log2_lambda);
           row_ok = row_ok && ok_r;
+          skip_r[rr] = ok_r;
         }
         skip = __all_sync(0xffffffffu, row_ok) != 0;
-        if (!skip) {
-          m_true[0] = fmaxf(m_true[0], r[0]);
-          m_true[1] = fmaxf(m_true[1], r[1]);
+        if (p.per_head) {
+          // Each query head is its own unit. A row that drops the tile gets zero
+          // probabilities; its tile maximum lies below its running maximum by
+          // -log2(lambda) > 0, so it cannot raise the reference either. The V
+          // rows are still loaded: the group's other heads may keep them.
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr)
+            if (!skip_r[rr]) m_true[rr] = fmaxf(m_true[rr], r[rr]);
+          if (p.skip_mask && warp == 0 && tq == 0) {
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const int row = g + 8 * rr;
+              if (row < G)
+                p.skip_mask[(size_t(seq) * p.Hq + kvh * G + row) * p.max_tiles + t0 / kDecTile] = skip_r[rr] ? 1 : 0;
+            }
+          }
+        } else {
+          skip_r[0] = skip_r[1] = false;
+          if (!skip) {
+            m_true[0] = fmaxf(m_true[0], r[0]);
+            m_true[1] = fmaxf(m_true[1], r[1]);
+          }
+          if (p.skip_mask && warp == 0 && lane == 0)
+            p.skip_mask[(size_t(seq) * p.Hkv + kvh) * p.max_tiles + t0 / kDecTile] = skip ? 1 : 0;
         }
-        if (p.skip_mask && warp == 0 && lane == 0)
-          p.skip_mask[(size_t(seq) * p.Hkv + kvh) * p.max_tiles + t0 / kDecTile] = skip ? 1 : 0;
       }
 
       if (!skip) {
@@ -444,10 +466,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           float pr[2][4];
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            pr[j][0] = row0_valid ? fast_exp2(s[j][0] - off0) : 0.f;
-            pr[j][1] = row0_valid ? fast_exp2(s[j][1] - off0) : 0.f;
-            pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
-            pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
+            pr[j][0] = (row0_valid && !skip_r[0]) ? fast_exp2(s[j][0] - off0) : 0.f;
+            pr[j][1] = (row0_valid && !skip_r[0]) ? fast_exp2(s[j][1] - off0) : 0.f;
+            pr[j][2] = (row1_valid && !skip_r[1]) ? fast_exp2(s[j][2] - off1) : 0.f;
+            pr[j][3] = (row1_valid && !skip_r[1]) ? fast_exp2(s[j][3] - off1) : 0.f;
           }
           pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
           pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);

@@ -184,6 +184,28 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                       uint8_t* skip_mask, int* device_status, void* stream);
 
 /*
+ * attn_decode_paged_blasst_heads -- attn_decode_paged with the BLASST tile skip
+ * ("高效部署稀疏注意力加速方案：BLASST方法详解与实践指南", section 架构与组件)
+ * decided for each query head alone: the unit is (sequence, query head, split)
+ * instead of the G heads that share a KV head. The page states the rule for
+ * the rows of a tile without fixing which rows share a tile in decode; this is
+ * the narrowest reading. A head that drops a 64-token tile gets no probability
+ * mass from it; the tile's K and V are still read while another head of the
+ * group keeps it.
+ * Arguments as attn_decode_paged, except:
+ *   skip_mask    [num_seqs][Hq][ceil(max_pages_per_seq*page_size/64)] uint8, may be
+ *                NULL: 1 skipped / 0 kept for every visited (head, tile)
+ *   lambda       in [0, 1); 0 decides nothing away (the dense result)
+ */
+int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const void* v_pages,
+                                   const int32_t* block_table, const int32_t* seq_lens,
+                                   int num_seqs, int Hq, int Hkv, int D, int page_size,
+                                   int max_pages_per_seq, int num_pages, float scale, float lambda,
+                                   int split_tokens, void* o, float* lse,
+                                   void* workspace, size_t workspace_bytes,
+                                   uint8_t* skip_mask, int* device_status, void* stream);
+
+/*
  * attn_decode_paged_noalloc -- attn_decode_paged without a caller-provided
  * workspace. (Library plumbing: the pages describe no counterpart.)
  *

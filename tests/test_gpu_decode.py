@@ -128,3 +128,39 @@ def test_decode_bad_page_raises_device_status(cuda_device):
     o_ref, lse_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens,
                                       16, gen.attn_scale(128), seqs=[0, 3])
     compare_output(o[[0, 3]], o_ref[[0, 3]], lse[[0, 3]], lse_ref[[0, 3]])
+
+
+@pytest.mark.parametrize("split", [256, 2048])
+@pytest.mark.parametrize("lam", [0.1, 0.3])
+def test_decode_blasst_per_head_matches_oracle(cuda_device, split, lam):
+    S, Hq, Hkv, D = 4096, 32, 8, 128
+    q, k, v = gen.peaked_prefill_inputs(1, Hq, Hkv, S, D, seed=2400, amp=8.0, period=split)
+    cache = gen.paged_from_contiguous(q[:, S - 1], k, v, page_size=16, seed=2401)
+    args = [t.to(cuda_device) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    scale = gen.attn_scale(D)
+    o, lse, mask = ab.decode_paged_blasst(*args, lam, scale=scale, split_tokens=split, rows_per_unit="head")
+    torch.cuda.synchronize()
+    assert mask.shape[1] == Hq
+    o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages,
+                                                            cache.block_table, cache.seq_lens, 16, scale, lam,
+                                                            split, rows_per_unit="head")
+    st = compare_skip(mask, m_ref, margin, label=f"per-head skip lam={lam}")
+    assert st["skipped"] > 0
+    if st["tie_mismatches"] == 0:
+        compare_output(o, o_ref, lse, lse_ref, label=f"per-head blasst lam={lam}")
+    # a head-level unit drops at least what its group drops
+    _, _, mg, _ = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages, cache.block_table,
+                                          cache.seq_lens, 16, scale, lam, split)
+    assert (m_ref == 1).sum() >= (mg == 1).sum() * (Hq // Hkv)
+
+
+def test_decode_blasst_per_head_lambda_zero_is_dense(cuda_device):
+    cache = gen.paged_decode_inputs(6, 32, 8, 128, 16, 64, 1500, seed=2450)
+    o0, l0, _, scale = _run(cache, cuda_device, 512)
+    args = [t.to(cuda_device) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    o1, l1, mask = ab.decode_paged_blasst(*args, 0.0, scale=scale, split_tokens=512, rows_per_unit="head")
+    torch.cuda.synchronize()
+    assert not (mask == 1).any()
+    o_ref, l_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens, 16,
+                                    scale)
+    compare_output(o1, o_ref, l1, l_ref, label="per-head lambda 0")
