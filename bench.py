@@ -457,6 +457,13 @@ def blasst_long_context_report(dev, reps=3):
             "ms": dms, "gbs_dense_equiv": dbytes / (dms * 1e-3) / 1e9,
             "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
             "max_abs_err_vs_dense": float(derr.max().item()), "speedup_vs_dense": dms0 / dms}
+        hms, (ho, hl, hmask) = timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split,
+                                                                    rows_per_unit="head"))
+        hvis = (hmask != 2)
+        report["decode"][str(lam) + "_per_head"] = {
+            "ms": hms, "skipped_frac": float(((hmask == 1) & hvis).sum().item() / hvis.sum().item()),
+            "max_abs_err_vs_dense": float((ho.float() - do0.float()).abs().max().item()),
+            "speedup_vs_dense": dms0 / hms}
 
     # The recipe above puts a raised key in every 64-key tile, so no tile can be
     # dropped. A second input with a single dominant key at position 0 (12 u on
