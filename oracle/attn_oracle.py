@@ -39,6 +39,7 @@ What it computes, and the passages it follows:
 
 * Chunked prefill over the paged cache (prefill_paged): the reading of
   "chunked prefill" stated in its docstring.
+* Writing new tokens' K/V into the paged cache (kv_append).
 
 Parity status: dense prefill, paged decode, chunked paged prefill and the
 gather are pinned by the
@@ -173,6 +174,41 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, page_size: int, sca
             ob, lb = attention_rows(q[b, hq][None, :], kb[:, kv, :], vb[:, kv, :], scale)
             o[b, hq], lse[b, hq] = ob[0], lb[0]
     return o, lse
+
+
+def kv_append(k_pages, v_pages, block_table, start_pos, k_new, v_new, page_size: int):
+    """Write the keys and values of new tokens into the paged cache.
+
+    The cache keeps the K/V of past tokens so that each new token only adds
+    its own ("TensorRT-LLM：大模型推理优化利器", section 4 on the KV cache; "LLM推理
+    优化技术综述", PART01), in fixed-size pages addressed through a block table
+    ("TensorRT对Grouped Query Attention的支持进展", section 动态形状与KV Cache管理).
+    Token t of sequence b goes to position p = start_pos[b] + t, that is to
+    physical page block_table[b][p // page_size], slot p % page_size.
+
+    k_pages/v_pages [P, page_size, Hkv, D]; k_new/v_new [N, T, Hkv, D]. Returns
+    new (k_pages, v_pages) numpy arrays in the input dtype's values (copies;
+    every other slot unchanged). Raises IndexError for a position past the
+    table or a page outside the pool.
+    """
+    def host(x):
+        return x.detach().cpu().float().numpy().copy() if hasattr(x, "detach") else np.array(x, copy=True)
+    kp, vp, kn, vn = host(k_pages), host(v_pages), host(k_new), host(v_new)
+    bt = np.asarray(block_table)
+    starts = np.asarray(start_pos)
+    N, T = kn.shape[0], kn.shape[1]
+    for b in range(N):
+        for t in range(T):
+            pos = int(starts[b]) + t
+            lp = pos // page_size
+            if lp >= bt.shape[1]:
+                raise IndexError(f"sequence {b}: position {pos} past the block table")
+            page = int(bt[b, lp])
+            if page < 0 or page >= kp.shape[0]:
+                raise IndexError(f"sequence {b}: block_table entry {page} out of range")
+            kp[page, pos % page_size] = kn[b, t]
+            vp[page, pos % page_size] = vn[b, t]
+    return kp, vp
 
 
 def prefill_paged(q, k_pages, v_pages, block_table, seq_lens, page_size: int, scale: float,

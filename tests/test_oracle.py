@@ -515,3 +515,48 @@ def test_prefill_paged_rejects_short_cache():
     with pytest.raises(ValueError):
         orc.prefill_paged(c.q, c.k_pages, c.v_pages, c.block_table, torch.tensor([3]), 16, 0.3)
 
+
+# ---------------------------------------------------------------- KV append
+
+def test_kv_append_then_gather_is_concatenation():
+    c = gen.paged_prefill_inputs(3, 1, 4, 2, 8, 16, [5, 16, 33], seed=37, poison=False)
+    g = torch.Generator().manual_seed(38)
+    T = 20
+    lens = [int(x) for x in c.seq_lens]
+    # room for T more tokens: extend the block tables with fresh pages
+    need = [-(-(L + T) // 16) for L in lens]
+    P0 = c.k_pages.shape[0]
+    extra = sum(max(0, n - -(-L // 16)) for n, L in zip(need, lens))
+    kp = torch.cat([c.k_pages, torch.zeros(extra, 16, 2, 8, dtype=torch.bfloat16)])
+    vp = torch.cat([c.v_pages, torch.zeros(extra, 16, 2, 8, dtype=torch.bfloat16)])
+    bt = torch.full((3, max(need)), -1, dtype=torch.int32)
+    nxt = P0
+    for b in range(3):
+        have = -(-lens[b] // 16)
+        bt[b, :have] = c.block_table[b, :have]
+        for j in range(have, need[b]):
+            bt[b, j] = nxt
+            nxt += 1
+    kn = torch.randn(3, T, 2, 8, generator=g).to(torch.bfloat16)
+    vn = torch.randn(3, T, 2, 8, generator=g).to(torch.bfloat16)
+    kp2, vp2 = orc.kv_append(kp, vp, bt, lens, kn, vn, 16)
+    for b in range(3):
+        kk = orc.gather_pages(kp2, bt[b].numpy(), lens[b] + T, 16)
+        vv = orc.gather_pages(vp2, bt[b].numpy(), lens[b] + T, 16)
+        np.testing.assert_array_equal(kk[:lens[b]], c.k_seqs[b].double().numpy())
+        np.testing.assert_array_equal(kk[lens[b]:], kn[b].double().numpy())
+        np.testing.assert_array_equal(vv[lens[b]:], vn[b].double().numpy())
+    # slots nobody wrote are unchanged
+    written = np.zeros(kp.shape[:2], dtype=bool)
+    for b in range(3):
+        for pos in range(lens[b] + T):
+            written[int(bt[b, pos // 16]), pos % 16] = True
+    np.testing.assert_array_equal(kp2[~written], kp.float().numpy()[~written])
+
+
+def test_kv_append_rejects_positions_past_the_table():
+    kp = np.zeros((4, 16, 1, 8))
+    bt = np.array([[0, 1]])
+    with pytest.raises(IndexError):
+        orc.kv_append(kp, kp, bt, [30], np.zeros((1, 3, 1, 8)), np.zeros((1, 3, 1, 8)), 16)
+
