@@ -51,6 +51,7 @@ SIGNATURES = {
                                _P, _SZ, _P, _P, _P]),
     "attn_decode_paged_blasst_heads": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P,
                                             _P, _P, _SZ, _P, _P, _P]),
+    "attn_kv_append": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                        _P, _P, _P]),
     "attn_read_device_status": (_I, [ctypes.POINTER(_I), _I]),
@@ -161,6 +162,23 @@ def prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float | Non
         Hkv, D, page_size, block_table.shape[1], P, scale, _ptr(device_status), _stream_handle(stream))
     _check(st, "attn_prefill_paged")
     return o, lse
+
+
+def kv_append(k_new, v_new, k_pages, v_pages, block_table, start_pos, device_status=None, stream=None):
+    """Write new tokens' K/V ([N,T,Hkv,D] bf16) into the page pools in place:
+    token t of sequence b goes to position start_pos[b] + t through block_table."""
+    _need(k_new, torch.bfloat16, 4, "k_new")
+    _need(v_new, torch.bfloat16, 4, "v_new")
+    _need(k_pages, torch.bfloat16, 4, "k_pages")
+    _need(v_pages, torch.bfloat16, 4, "v_pages")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(start_pos, torch.int32, 1, "start_pos")
+    N, T, Hkv, D = k_new.shape
+    P, page_size, _, _ = k_pages.shape
+    st = load_library().attn_kv_append(
+        _ptr(k_new), _ptr(v_new), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(start_pos), N, T, Hkv, D,
+        page_size, block_table.shape[1], P, _ptr(device_status), _stream_handle(stream))
+    _check(st, "attn_kv_append")
 
 
 def prefill_skip_mask_shape(B, Hq, S):

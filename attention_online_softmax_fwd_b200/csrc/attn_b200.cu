@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_heads.cuh"
+#include "kv_append.cuh"
 #include "prefill.cuh"
 
 using namespace attn;
@@ -422,6 +423,37 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
                     : dispatch_decode_g<128, false>(G, tk, tv, p, sms, s);
   return use_skip ? dispatch_decode_g<64, true>(G, tk, tv, p, sms, s)
                   : dispatch_decode_g<64, false>(G, tk, tv, p, sms, s);
+}
+
+int attn_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages, const int32_t* block_table,
+                   const int32_t* start_pos, int num_seqs, int T, int Hkv, int D, int page_size,
+                   int max_pages_per_seq, int num_pages, int* device_status, void* stream) {
+  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !start_pos) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pages) || !aligned16(v_pages))
+    return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(start_pos) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (num_seqs < 1 || T < 1 || Hkv < 1) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!valid_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+  if ((long long)num_seqs * T > (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  int sms = 0;
+  if (int st = current_device(&sms)) return st;
+  KvAppendParams p{};
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_pages = static_cast<__nv_bfloat16*>(k_pages);
+  p.v_pages = static_cast<__nv_bfloat16*>(v_pages);
+  p.block_table = block_table;
+  p.start_pos = start_pos;
+  p.status = device_status;
+  p.N = num_seqs; p.T = T; p.Hkv = Hkv; p.D = D;
+  p.page_size = page_size; p.max_pages = max_pages_per_seq; p.num_pages = num_pages;
+  const long long rows = (long long)num_seqs * T;
+  long long blocks = (rows + 7) / 8;   // eight warps per block, one token row each
+  if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
+  kv_append_kernel<<<dim3(unsigned(blocks)), dim3(256), 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
 }
 
 int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,

@@ -133,6 +133,29 @@ int attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
                        int* device_status, void* stream);
 
 /*
+ * attn_kv_append -- write the keys and values of new tokens into the paged
+ * cache ("TensorRT-LLM：大模型推理优化利器", section 4: the cache keeps the K/V
+ * of past tokens; "TensorRT对Grouped Query Attention的支持进展", section 动态形状
+ * 与KV Cache管理: fixed-size pages addressed through physical page indices).
+ * Token t of sequence b goes to position start_pos[b] + t, i.e. page
+ * block_table[b][pos / page_size], slot pos % page_size; nothing else is
+ * written. Run it before attn_decode_paged / attn_prefill_paged on the same
+ * stream, with seq_lens then covering the new tokens.
+ *   k_new, v_new  [num_seqs][T][Hkv][D] bf16 (16-byte aligned)
+ *   k_pages,
+ *   v_pages       [num_pages][page_size][Hkv][D] bf16, written in place
+ *   block_table   [num_seqs][max_pages_per_seq] int32 (device)
+ *   start_pos     [num_seqs] int32 (device): cached tokens before the append
+ *   device_status may be NULL; a position past the table or a page outside
+ *                 [0, num_pages) is skipped and ATTN_ERR_DEVICE_BOUNDS set
+ * D 64 or 128; page_size 16, 32, 64, 128 or 256. Errors as attn_prefill.
+ */
+int attn_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                   const int32_t* block_table, const int32_t* start_pos, int num_seqs, int T,
+                   int Hkv, int D, int page_size, int max_pages_per_seq, int num_pages,
+                   int* device_status, void* stream);
+
+/*
  * attn_decode_workspace_bytes -- scratch needed by attn_decode_paged.
  * The decode splits each sequence's keys into chunks of split_tokens tokens,
  * computes one partial (O, LSE) per (sequence, query head, chunk), and merges

@@ -143,3 +143,21 @@ def test_prefill_paged_rejects_bad_arguments(lib, bad):
 
 def test_prefill_paged_rejects_unsupported_head_dim(lib):
     assert _paged_prefill(lib, D=96) == UNSUPPORTED
+
+
+def _append(lib, **kw):
+    a = dict(kn=FAKE, vn=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sp=FAKE, N=4, T=1, Hkv=8, D=128, ps=16, mp=8, P=64)
+    a.update(kw)
+    return lib.attn_kv_append(a["kn"], a["vn"], a["kp"], a["vp"], a["bt"], a["sp"], a["N"], a["T"], a["Hkv"],
+                              a["D"], a["ps"], a["mp"], a["P"], None, None)
+
+
+@pytest.mark.parametrize("bad", [dict(kn=None), dict(vp=None), dict(bt=None), dict(sp=None),
+                                 dict(kn=ctypes.c_void_p((1 << 20) + 8)), dict(sp=ctypes.c_void_p((1 << 20) + 1)),
+                                 dict(N=0), dict(T=0), dict(Hkv=0), dict(ps=24), dict(mp=0), dict(P=0)])
+def test_kv_append_rejects_bad_arguments(lib, bad):
+    assert _append(lib, **bad) == INVALID
+
+
+def test_kv_append_rejects_unsupported_head_dim(lib):
+    assert _append(lib, D=80) == UNSUPPORTED
