@@ -158,6 +158,18 @@ def paged_prefill_inputs(B, Sq, Hq, Hkv, D, page_size, lens, seed, poison=True, 
                         k_seqs, v_seqs, page_size)
 
 
+def quantize_pool_e4m3(pool):
+    """FP8 E4M3 codes (uint8, same shape) and the scale of a bf16 page pool:
+    scale = max|finite x| / 448, codes = e4m3(x / scale) rounded to nearest
+    (NaN stays NaN)."""
+    x = pool.float()
+    finite = torch.isfinite(x)
+    amax = float(x[finite].abs().max()) if finite.any() else 1.0
+    scale = max(amax, 1e-30) / 448.0
+    codes = (x / scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, scale
+
+
 # The workloads the library is measured and checked on (sizes as named).
 CONFIGS = {
     "tiny_gqa_prefill": dict(kind="prefill", B=1, Hq=4, Hkv=2, S=128, D=64, causal=True, seed=1001),

@@ -40,6 +40,8 @@ What it computes, and the passages it follows:
 * Chunked prefill over the paged cache (prefill_paged): the reading of
   "chunked prefill" stated in its docstring.
 * Writing new tokens' K/V into the paged cache (kv_append).
+* FP8 E4M3 paged cache with one scale per pool (decode_paged_fp8): the
+  reading stated in its docstring; E4M3 decoded from its bit layout.
 
 Parity status: dense prefill, paged decode, chunked paged prefill and the
 gather are pinned by the
@@ -250,6 +252,37 @@ def prefill_paged(q, k_pages, v_pages, block_table, seq_lens, page_size: int, sc
             o[b, :, hq, :] = ob
             lse[b, hq, :] = lb
     return o, lse
+
+
+def e4m3_to_float(codes):
+    """Float64 values of FP8 E4M3 codes (uint8): 1 sign bit, 4 exponent bits with
+    bias 7, 3 mantissa bits; exponent 0 holds the subnormals m/8 * 2^-6; no
+    infinities, and S.1111.111 is NaN (so the largest finite value is 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    val = sign * val
+    return np.where((c & 0x7F) == 0x7F, np.nan, val)
+
+
+def decode_paged_fp8(q, k_codes, v_codes, k_scale: float, v_scale: float, block_table, seq_lens,
+                     page_size: int, scale: float, seqs=None):
+    """Single-token decode over a paged cache stored as FP8 E4M3.
+
+    The TensorRT-LLM page ("TensorRT-LLM：大模型推理优化利器", 量化) lists FP8
+    among the low-precision formats for cutting memory and bandwidth, and the
+    integration page ("flash-attention与TensorRT-LLM集成") stores in FP8. The
+    scale convention is not given; the reading used: one scale per pool,
+    K = k_scale * e4m3(k_codes) and V = v_scale * e4m3(v_codes). The oracle
+    dequantises the codes it gathers and applies the dense decode.
+
+    k_codes/v_codes [P, page_size, Hkv, D] uint8; other arguments as decode_paged.
+    """
+    k = e4m3_to_float(np.asarray(k_codes.cpu() if hasattr(k_codes, "cpu") else k_codes)) * float(k_scale)
+    v = e4m3_to_float(np.asarray(v_codes.cpu() if hasattr(v_codes, "cpu") else v_codes)) * float(v_scale)
+    return decode_paged(q, k, v, block_table, seq_lens, page_size, scale, seqs=seqs)
 
 
 # ----------------------------------------------------------------------------

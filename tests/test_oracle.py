@@ -560,3 +560,36 @@ def test_kv_append_rejects_positions_past_the_table():
     with pytest.raises(IndexError):
         orc.kv_append(kp, kp, bt, [30], np.zeros((1, 3, 1, 8)), np.zeros((1, 3, 1, 8)), 16)
 
+
+# ---------------------------------------------------------------- FP8 cache
+
+def test_e4m3_decoding_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = orc.e4m3_to_float(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    np.testing.assert_array_equal(ours[~np.isnan(ours)], ref[~np.isnan(ref)])
+    assert np.nanmax(ours) == 448.0 and np.nanmin(ours[ours > 0]) == 2.0 ** -9
+
+
+def test_quantised_pool_within_half_an_e4m3_step():
+    c = gen.paged_decode_inputs(4, 8, 2, 64, 16, 30, 90, seed=39, poison=False)
+    codes, s = gen.quantize_pool_e4m3(c.k_pages)
+    x = c.k_pages.double().numpy()
+    deq = orc.e4m3_to_float(codes.numpy()) * s
+    # round to nearest: |error| <= 2^-4 |x| for normals, <= 2^-10 * s for subnormals
+    assert (np.abs(deq - x) <= np.maximum(np.abs(x) * 2.0 ** -4, s * 2.0 ** -10) + 1e-12).all()
+
+
+def test_fp8_decode_is_decode_of_the_dequantised_cache():
+    c = gen.paged_decode_inputs(3, 8, 2, 64, 16, 20, 200, seed=40)
+    kc, ks = gen.quantize_pool_e4m3(c.k_pages)
+    vc, vs = gen.quantize_pool_e4m3(c.v_pages)
+    o, lse = orc.decode_paged_fp8(c.q, kc, vc, ks, vs, c.block_table, c.seq_lens, 16, 0.3)
+    kd = orc.e4m3_to_float(kc.numpy()) * ks
+    vd = orc.e4m3_to_float(vc.numpy()) * vs
+    od, ld = orc.decode_paged(c.q, kd, vd, c.block_table, c.seq_lens, 16, 0.3)
+    np.testing.assert_array_equal(o, od)
+    np.testing.assert_array_equal(lse, ld)
+    assert np.isfinite(o).all()                   # poisoned (NaN) slots are never read
+
