@@ -8,5 +8,5 @@ synthetic workloads.
 
 from .binding import (  # noqa: F401
     AttnError, decode_paged, decode_paged_blasst, decode_workspace_bytes, lib_path,
-    kv_append, load_library, prefill, prefill_blasst, prefill_paged,
+    decode_paged_fp8, kv_append, load_library, prefill, prefill_blasst, prefill_paged,
 )

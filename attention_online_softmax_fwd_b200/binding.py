@@ -52,6 +52,8 @@ SIGNATURES = {
     "attn_decode_paged_blasst_heads": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P,
                                             _P, _P, _SZ, _P, _P, _P]),
     "attn_kv_append": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "attn_decode_paged_fp8": (_I, [_P, _P, _P, _F, _F, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P,
+                                   _P, _SZ, _P, _P]),
     "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                        _P, _P, _P]),
     "attn_read_device_status": (_I, [ctypes.POINTER(_I), _I]),
@@ -270,6 +272,40 @@ def decode_paged_blasst(q, k_pages, v_pages, block_table, seq_lens, lam: float, 
         raise AttnError("rows_per_unit must be 'group' or 'head'")
     return _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens, out, lse,
                    workspace, skip_mask, device_status, return_lse, stream, per_head=rows_per_unit == "head")
+
+
+def decode_paged_fp8(q, k_codes, v_codes, k_scale: float, v_scale: float, block_table, seq_lens, scale=None,
+                     split_tokens: int = 1024, out=None, lse=None, workspace=None, device_status=None,
+                     return_lse=True, stream=None):
+    """Dense paged decode over FP8 E4M3 code pools (uint8 [P, page_size, Hkv, D]) with
+    one scale per pool: K = k_scale * e4m3(k_codes), V = v_scale * e4m3(v_codes).
+    Returns (o [N,Hq,D] bf16, lse [N,Hq] fp32)."""
+    _need(q, torch.bfloat16, 3, "q")
+    _need(k_codes, torch.uint8, 4, "k_codes")
+    _need(v_codes, torch.uint8, 4, "v_codes")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    N, Hq, D = q.shape
+    P, page_size, Hkv, Dk = k_codes.shape
+    if v_codes.shape != k_codes.shape or Dk != D or block_table.shape[0] != N or seq_lens.shape[0] != N:
+        raise AttnError("inconsistent decode shapes")
+    max_pages = block_table.shape[1]
+    scale = default_scale(D) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    if lse is None and return_lse:
+        lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(N, Hq, D, max_pages, page_size, split_tokens)
+    if need == 0:
+        raise AttnError("invalid decode configuration", 1)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = load_library().attn_decode_paged_fp8(
+        _ptr(q), _ptr(k_codes), _ptr(v_codes), float(k_scale), float(v_scale), _ptr(block_table),
+        _ptr(seq_lens), N, Hq, Hkv, D, page_size, max_pages, P, scale, split_tokens, _ptr(o), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(device_status),
+        _stream_handle(stream))
+    _check(st, "attn_decode_paged_fp8")
+    return o, lse
 
 
 def decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale=None, split_tokens: int = 1024,

@@ -63,16 +63,17 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 4-D bf16 tensor map. dims/box innermost first; strides in bytes for dims 1..3.
+// 4-D tensor map (bf16 unless told otherwise). dims/box innermost first; strides in bytes for dims 1..3.
 int encode_map(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
-               const uint32_t box[4], CUtensorMapSwizzle swizzle) {
+               const uint32_t box[4], CUtensorMapSwizzle swizzle,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensor_map_encoder();
   if (!enc) return ATTN_ERR_CUDA;
   const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
   cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
   cuuint64_t s[3] = {strides[0], strides[1], strides[2]};
   cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d, s, b, elem_strides,
+  const CUresult r = enc(map, dtype, 4, const_cast<void*>(base), d, s, b, elem_strides,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
@@ -227,11 +228,11 @@ int dispatch_decode_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const
   }
 }
 
-template <int D, int G, int HG>
+template <int D, int G, int HG, bool F8 = false>
 int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int* ticket_counter,
                         int sms, cudaStream_t stream) {
-  auto kernel = decode_heads_kernel<D, G, HG>;
-  constexpr int smem = DecodeHeadsSmem<D, G, HG>::kDynamic;
+  auto kernel = decode_heads_kernel<D, G, HG, F8>;
+  constexpr int smem = DecodeHeadsSmem<D, G, HG, F8>::kDynamic;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
@@ -241,24 +242,24 @@ int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
   return launch_merge<D>(p, stream);
 }
 
-template <int D, int HG>
+template <int D, int HG, bool F8 = false>
 int dispatch_decode_heads_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int* ctr,
                             int sms, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_decode_heads<D, 1, HG>(tk, tv, p, ctr, sms, s);
-    case 2: return launch_decode_heads<D, 2, HG>(tk, tv, p, ctr, sms, s);
-    case 4: return launch_decode_heads<D, 4, HG>(tk, tv, p, ctr, sms, s);
-    case 8: return launch_decode_heads<D, 8, HG>(tk, tv, p, ctr, sms, s);
-    case 16: return launch_decode_heads<D, 16, HG>(tk, tv, p, ctr, sms, s);
+    case 1: return launch_decode_heads<D, 1, HG, F8>(tk, tv, p, ctr, sms, s);
+    case 2: return launch_decode_heads<D, 2, HG, F8>(tk, tv, p, ctr, sms, s);
+    case 4: return launch_decode_heads<D, 4, HG, F8>(tk, tv, p, ctr, sms, s);
+    case 8: return launch_decode_heads<D, 8, HG, F8>(tk, tv, p, ctr, sms, s);
+    case 16: return launch_decode_heads<D, 16, HG, F8>(tk, tv, p, ctr, sms, s);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
 
-template <int D>
+template <int D, bool F8 = false>
 int dispatch_decode_heads(int G, int hg, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           int* ctr, int sms, cudaStream_t s) {
-  return hg == 8 ? dispatch_decode_heads_g<D, 8>(G, tk, tv, p, ctr, sms, s)
-                 : dispatch_decode_heads_g<D, 4>(G, tk, tv, p, ctr, sms, s);
+  return hg == 8 ? dispatch_decode_heads_g<D, 8, F8>(G, tk, tv, p, ctr, sms, s)
+                 : dispatch_decode_heads_g<D, 4, F8>(G, tk, tv, p, ctr, sms, s);
 }
 
 }  // namespace
@@ -474,6 +475,75 @@ int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const voi
   return decode_impl(q, k_pages, v_pages, block_table, seq_lens, num_seqs, Hq, Hkv, D, page_size,
                      max_pages_per_seq, num_pages, scale, lambda, split_tokens, o, lse, workspace, workspace_bytes,
                      skip_mask, device_status, stream, true);
+}
+
+int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_codes, float k_scale, float v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D,
+                          int page_size, int max_pages_per_seq, int num_pages, float scale, int split_tokens,
+                          void* o, float* lse, void* workspace, size_t workspace_bytes, int* device_status,
+                          void* stream) {
+  if (!q || !k_codes || !v_codes || !block_table || !seq_lens || !o || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(o) || !aligned16(workspace))
+    return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (num_seqs < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!valid_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+  if (split_tokens < 64 || split_tokens % 64 != 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(k_scale) || !(k_scale > 0.f) || !std::isfinite(v_scale) || !(v_scale > 0.f))
+    return ATTN_ERR_INVALID_ARG;
+  if ((long long)max_pages_per_seq * page_size > (1ll << 30)) return ATTN_ERR_INVALID_ARG;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return ATTN_ERR_UNSUPPORTED;
+  const int hg = Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0);
+  if (hg == 0) return ATTN_ERR_UNSUPPORTED;
+  const size_t need = attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens);
+  if (need == 0 || workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
+  const float scale_log2 = scale * k_scale * 1.4426950408889634f;
+  if (!std::isfinite(scale_log2) || !(scale_log2 > 0.f)) return ATTN_ERR_INVALID_ARG;
+  int sms = 0;
+  if (int st = current_device(&sms)) return st;
+
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
+  int* ticket_counter = static_cast<int*>(workspace);
+  p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader);
+  const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader + (o_bytes + 255) / 256 * 256);
+  p.status = device_status;
+  p.num_seqs = num_seqs; p.Hq = Hq; p.Hkv = Hkv;
+  p.page_size = page_size; p.max_pages = max_pages_per_seq; p.num_pages = num_pages;
+  p.split_tokens = split_tokens;
+  p.max_splits = int(ms);
+  p.max_tiles = int(((long long)max_pages_per_seq * page_size + 63) / 64);
+  p.chunk = page_size < 64 ? page_size : 64;
+  p.scale_log2 = scale_log2;
+  p.log2_lambda = -INFINITY;
+  p.v_scale = v_scale;
+  p.num_items = (long long)num_seqs * ms * Hkv;
+
+  // code pool [P][page_size][Hkv][128] as a 4-D map {128, page_size, Hkv, P}; box = 16 slots of hg
+  // heads, each head's slots one 2 KB block of 128-byte rows under the 128-byte swizzle
+  const uint64_t dims[4] = {uint64_t(D), uint64_t(page_size), uint64_t(Hkv), uint64_t(num_pages)};
+  const uint64_t strides[3] = {uint64_t(Hkv) * D, uint64_t(D), uint64_t(page_size) * Hkv * D};
+  const uint32_t box[4] = {uint32_t(D), uint32_t(kDhChunk), uint32_t(hg), 1};
+  CUtensorMap hk, hv;
+  if (int st = encode_map(&hk, k_codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_DATA_TYPE_UINT8))
+    return st;
+  if (int st = encode_map(&hv, v_codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_DATA_TYPE_UINT8))
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ticket_counter, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+  return dispatch_decode_heads<128, true>(G, hg, hk, hv, p, ticket_counter, sms, s);
 }
 
 }  // extern "C"

@@ -45,6 +45,7 @@ struct DecodeParams {
   int chunk;          // tokens per TMA copy: min(page_size, 64)
   float scale_log2;   // softmax scale * log2(e)
   float log2_lambda;  // log2(lambda) for the tile skip
+  float v_scale;      // FP8 cache: V = v_scale * code (the K scale is folded into scale_log2)
   int per_head;       // tile skip decided for each query head alone, not for the KV head's group
   long long num_items;
 };

@@ -14,6 +14,23 @@
 // runs the online softmax in its accumulator registers across the whole item,
 // and writes the item's result for its heads at the end -- no cross-warp merge.
 // Split partials are combined by decode_merge_kernel as in the per-head path.
+//
+// F8 = true reads a cache stored as FP8 E4M3 codes with one scale per pool
+// (K = k_scale * code, V = v_scale * code; k_scale is folded into the score
+// scale and v_scale into the output normalisation on the host). A head's 16
+// tokens are then one 2 KB block of 128-byte rows (D = 128). The codes go from
+// shared memory straight into mma fragments, widened to f16 on the way (exact),
+// and the query rows are taken to f16 once per item:
+//   * q K^T: the head dimension is summed over, so it may be visited in any
+//     order that q and K share. Lane (g, t) loads bytes [32t, 32t + 32) of key
+//     row g; in k-step ks its fragment halves hold bytes 32t + 4ks + {0, 1} and
+//     32t + 4ks + {2, 3}, and its q fragments take the same dimensions.
+//   * P V: output column c of n-tile n is head dimension 16c + n, so lane
+//     (g, t) loads byte group g (dims 16g .. 16g + 15) of the token rows it
+//     needs, pairs the bytes of two tokens with a byte permute, and ends up
+//     owning output dims 32t .. 32t + 31 (o[n][0] = dim 32t + n,
+//     o[n][1] = dim 32t + 16 + n).
+// P is rounded to f16 for P V and the normaliser sums the rounded values.
 #pragma once
 
 #include "decode.cuh"
@@ -22,9 +39,9 @@ namespace attn {
 
 constexpr int kDhChunk = 16;  // tokens per stage
 
-template <int D, int G, int HG>
+template <int D, int G, int HG, bool F8 = false>
 struct DecodeHeadsSmem {
-  static constexpr int kHeadBytes = kDhChunk * D * 2;   // one head's 16 tokens
+  static constexpr int kHeadBytes = kDhChunk * D * (F8 ? 1 : 2);   // one head's 16 tokens
   static constexpr int kKVBytes = HG * kHeadBytes;      // K (or V) rows of one stage
   static constexpr int kQBytes = HG * G * D * 2;        // the item's query rows
   static constexpr int kStageBytes = (2 * kKVBytes + kQBytes + 1023) / 1024 * 1024;
@@ -50,12 +67,13 @@ __device__ __forceinline__ void dh_item_coords(long long item, int num_seqs, int
   grp = rem % n_groups;
 }
 
-template <int D, int G, int HG>
+template <int D, int G, int HG, bool F8 = false>
 __global__ void __launch_bounds__((HG + 1) * 32, 1)
     decode_heads_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeParams p, int* ticket_counter) {
   static_assert(G >= 1 && G <= 16, "query heads per KV head");
-  using L = DecodeHeadsSmem<D, G, HG>;
+  static_assert(!F8 || D == 128, "the FP8 cache layout assumes 128-byte rows");
+  using L = DecodeHeadsSmem<D, G, HG, F8>;
   constexpr int NS = L::kStages;
   constexpr int KS = D / 16;
   constexpr int NT = D / 8;
@@ -159,8 +177,13 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           if (first) bulk_load(stage + 2 * L::kKVBytes, qsrc, uint32_t(L::kQBytes), &full[slot]);
           if (valid) {
             const int in_page = t0 % p.page_size;
-            tma_load_5d(stage, &tm_k, &full[slot], 0, 0, in_page, grp * HG, page);
-            tma_load_5d(stage + L::kKVBytes, &tm_v, &full[slot], 0, 0, in_page, grp * HG, page);
+            if constexpr (F8) {
+              tma_load_4d(stage, &tm_k, &full[slot], 0, in_page, grp * HG, page);
+              tma_load_4d(stage + L::kKVBytes, &tm_v, &full[slot], 0, in_page, grp * HG, page);
+            } else {
+              tma_load_5d(stage, &tm_k, &full[slot], 0, 0, in_page, grp * HG, page);
+              tma_load_5d(stage + L::kKVBytes, &tm_v, &full[slot], 0, 0, in_page, grp * HG, page);
+            }
           }
         }
         __syncwarp();
@@ -211,12 +234,23 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         n_splits = (ti.len + p.split_tokens - 1) / p.split_tokens;
         const uint32_t* qs = reinterpret_cast<const uint32_t*>(stage + 2 * L::kKVBytes) + warp * G * (D / 2);
         const int h0 = row0_valid ? g : 0, h1 = row1_valid ? g + 8 : 0;
+        if constexpr (F8) {
+          // dims 32tq + 4ks + {0,1} and {2,3}, matching the key fragments below
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qa[ks][0] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + tq] : 0u;
-          qa[ks][1] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + tq] : 0u;
-          qa[ks][2] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + 4 + tq] : 0u;
-          qa[ks][3] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + 4 + tq] : 0u;
+          for (int ks = 0; ks < KS; ++ks) {
+            qa[ks][0] = row0_valid ? bf16x2_to_f16x2(qs[h0 * (D / 2) + 16 * tq + 2 * ks]) : 0u;
+            qa[ks][1] = row1_valid ? bf16x2_to_f16x2(qs[h1 * (D / 2) + 16 * tq + 2 * ks]) : 0u;
+            qa[ks][2] = row0_valid ? bf16x2_to_f16x2(qs[h0 * (D / 2) + 16 * tq + 2 * ks + 1]) : 0u;
+            qa[ks][3] = row1_valid ? bf16x2_to_f16x2(qs[h1 * (D / 2) + 16 * tq + 2 * ks + 1]) : 0u;
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            qa[ks][0] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + tq] : 0u;
+            qa[ks][1] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + tq] : 0u;
+            qa[ks][2] = row0_valid ? qs[h0 * (D / 2) + ks * 8 + 4 + tq] : 0u;
+            qa[ks][3] = row1_valid ? qs[h1 * (D / 2) + ks * 8 + 4 + tq] : 0u;
+          }
         }
 #pragma unroll
         for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -237,16 +271,34 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int a = 0; a < 2; ++a) sp[j][a][0] = sp[j][a][1] = sp[j][a][2] = sp[j][a][3] = 0.f;
-          const int mi = lane >> 3, r = lane & 7;
-          const int tok = (mi >> 1) * 8 + r;
-          uint32_t bfr[KS][4];
+          if constexpr (F8) {
+            // key row j*8 + g (its swizzle phase is g), bytes [32tq, 32tq + 32)
+            const uint8_t* kb = stage + warp * L::kHeadBytes;
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks)
-            ldsm_x4(kaddr + swz_off<D>(tok, ks * 2 + (mi & 1)), bfr[ks][0], bfr[ks][1], bfr[ks][2], bfr[ks][3]);
+            for (int j = 0; j < 2; ++j) {
+              const uint8_t* row = kb + (j * 8 + g) * 128;
+              const uint4 w0 = *reinterpret_cast<const uint4*>(row + (((2 * tq) ^ g) << 4));
+              const uint4 w1 = *reinterpret_cast<const uint4*>(row + (((2 * tq + 1) ^ g) << 4));
+              const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            mma_bf16_16816(sp[0][ks & 1], qa[ks], bfr[ks][0], bfr[ks][1]);
-            mma_bf16_16816(sp[1][ks & 1], qa[ks], bfr[ks][2], bfr[ks][3]);
+              for (int ks = 0; ks < KS; ++ks) {
+                uint32_t b0, b1;
+                e4m3x4_to_f16x2x2(w[ks], b0, b1);
+                mma_f16_16816(sp[j][ks & 1], qa[ks], b0, b1);
+              }
+            }
+          } else {
+            const int mi = lane >> 3, r = lane & 7;
+            const int tok = (mi >> 1) * 8 + r;
+            uint32_t bfr[KS][4];
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks)
+              ldsm_x4(kaddr + swz_off<D>(tok, ks * 2 + (mi & 1)), bfr[ks][0], bfr[ks][1], bfr[ks][2], bfr[ks][3]);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              mma_bf16_16816(sp[0][ks & 1], qa[ks], bfr[ks][0], bfr[ks][1]);
+              mma_bf16_16816(sp[1][ks & 1], qa[ks], bfr[ks][2], bfr[ks][3]);
+            }
           }
 #pragma unroll
           for (int j = 0; j < 2; ++j)
@@ -270,7 +322,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
           mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
         }
-        if (!clean) {
+        if (!F8 && !clean) {
           // zero the V rows of tokens past the end so that 0 * (stale or NaN) cannot reach O
           for (int t = ntok; t < kDhChunk; ++t)
             for (int c = lane; c < D / 8; c += 32)
@@ -311,20 +363,51 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
             pr[j][2] = row1_valid ? fast_exp2(s[j][2] - off1) : 0.f;
             pr[j][3] = row1_valid ? fast_exp2(s[j][3] - off1) : 0.f;
           }
-          pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-          pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-          pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-          pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
           l_part[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
           l_part[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
           // the weights applied to V are normalised by the sum of the rounded P, so
           // they add up to one (a dominant key's P, up to 2^8 under the lagging
-          // reference, would otherwise carry its bf16 rounding into the whole row)
-          lr_part[0] += (bf16_lo(pa[0]) + bf16_hi(pa[0])) + (bf16_lo(pa[2]) + bf16_hi(pa[2]));
-          lr_part[1] += (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));
+          // reference, would otherwise carry its rounding into the whole row)
+          if constexpr (F8) {
+            pa[0] = pack_f16x2(pr[0][0], pr[0][1]);
+            pa[1] = pack_f16x2(pr[0][2], pr[0][3]);
+            pa[2] = pack_f16x2(pr[1][0], pr[1][1]);
+            pa[3] = pack_f16x2(pr[1][2], pr[1][3]);
+            lr_part[0] += (f16_lo(pa[0]) + f16_hi(pa[0])) + (f16_lo(pa[2]) + f16_hi(pa[2]));
+            lr_part[1] += (f16_lo(pa[1]) + f16_hi(pa[1])) + (f16_lo(pa[3]) + f16_hi(pa[3]));
+          } else {
+            pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+            pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+            pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+            pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+            lr_part[0] += (bf16_lo(pa[0]) + bf16_hi(pa[0])) + (bf16_lo(pa[2]) + bf16_hi(pa[2]));
+            lr_part[1] += (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));
+          }
         }
         // ---- O += P V over the 16 tokens
-        {
+        if constexpr (F8) {
+          // token rows 2tq, 2tq + 1, 2tq + 8, 2tq + 9 (swizzle phases 2tq, 2tq + 1), byte group g;
+          // rows past the end are zeroed here so that 0 * (stale or NaN) cannot reach O
+          const uint8_t* vb = stage + L::kKVBytes + warp * L::kHeadBytes;
+          uint4 vr[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tok = 2 * tq + (i & 1) + (i >> 1) * 8;
+            vr[i] = *reinterpret_cast<const uint4*>(vb + tok * 128 + ((g ^ (tok & 7)) << 4));
+            if (!clean && tok >= ntok) vr[i] = make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t a = (&vr[0].x)[w], b = (&vr[1].x)[w], c = (&vr[2].x)[w], d = (&vr[3].x)[w];
+            uint32_t b0[4], b1[4];   // n-tile 4w + i: (token 2tq, 2tq + 1) and (2tq + 8, 2tq + 9)
+            e4m3x4_to_f16x2x2(__byte_perm(a, b, 0x5140), b0[0], b0[1]);
+            e4m3x4_to_f16x2x2(__byte_perm(a, b, 0x7362), b0[2], b0[3]);
+            e4m3x4_to_f16x2x2(__byte_perm(c, d, 0x5140), b1[0], b1[1]);
+            e4m3x4_to_f16x2x2(__byte_perm(c, d, 0x7362), b1[2], b1[3]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mma_f16_16816(o[4 * w + i], pa, b0[i], b1[i]);
+          }
+        } else {
           const int mi = lane >> 3, r = lane & 7;
           const int tok = (mi & 1) * 8 + r;
 #pragma unroll
@@ -335,7 +418,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
             mma_bf16_16816(o[2 * n2 + 1], pa, v2, v3);
           }
         }
-        if (!clean) fence_proxy_async_smem();   // zeroed rows before the next TMA write
+        if (!F8 && !clean) fence_proxy_async_smem();   // zeroed rows before the next TMA write
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
@@ -356,19 +439,47 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         if (!valid) continue;
         const int hq = (grp * HG + warp) * G + g + 8 * r;
         const float lsum = l_part[r];
-        const float inv = lr_part[r] > 0.f ? 1.f / lr_part[r] : 0.f;   // 0 only if every page was invalid
+        float inv = lr_part[r] > 0.f ? 1.f / lr_part[r] : 0.f;   // 0 only if every page was invalid
+        if constexpr (F8) inv *= p.v_scale;
         if (n_splits == 1) {
-          __nv_bfloat16* dst = p.o + (size_t(seq) * p.Hq + hq) * D + 2 * tq;
+          if constexpr (F8) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(seq) * p.Hq + hq) * D + 32 * tq);
 #pragma unroll
-          for (int n = 0; n < NT; ++n)
-            *reinterpret_cast<uint32_t*>(dst + n * 8) = pack_bf16x2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int q8 = 0; q8 < 2; ++q8) {
+                const int n = 8 * q8, e = 2 * r + h;
+                dst[2 * h + q8] = make_uint4(pack_bf16x2(o[n][e] * inv, o[n + 1][e] * inv),
+                                             pack_bf16x2(o[n + 2][e] * inv, o[n + 3][e] * inv),
+                                             pack_bf16x2(o[n + 4][e] * inv, o[n + 5][e] * inv),
+                                             pack_bf16x2(o[n + 6][e] * inv, o[n + 7][e] * inv));
+              }
+          } else {
+            __nv_bfloat16* dst = p.o + (size_t(seq) * p.Hq + hq) * D + 2 * tq;
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+              *reinterpret_cast<uint32_t*>(dst + n * 8) = pack_bf16x2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+          }
           if (p.lse && tq == 0)
             p.lse[size_t(seq) * p.Hq + hq] = lsum > 0.f ? (m_ref[r] + __log2f(lsum)) * 0.69314718055994531f : neg_inf;
         } else {
-          float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + 2 * tq;
+          if constexpr (F8) {
+            float4* dst = reinterpret_cast<float4*>(p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D +
+                                                    32 * tq);
 #pragma unroll
-          for (int n = 0; n < NT; ++n)
-            *reinterpret_cast<float2*>(dst + n * 8) = make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int n = 0; n < NT; n += 4) {
+                const int e = 2 * r + h;
+                dst[4 * h + n / 4] = make_float4(o[n][e] * inv, o[n + 1][e] * inv, o[n + 2][e] * inv,
+                                                 o[n + 3][e] * inv);
+              }
+          } else {
+            float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + 2 * tq;
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+              *reinterpret_cast<float2*>(dst + n * 8) = make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+          }
           if (tq == 0)
             p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lsum > 0.f ? m_ref[r] + __log2f(lsum) : neg_inf;
         }

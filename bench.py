@@ -47,11 +47,11 @@ def prefill_flops(B, Hq, S, D, causal=True):
     return 4.0 * D * B * Hq * pairs
 
 
-def decode_bytes(seq_lens, Hq, Hkv, D, max_pages):
+def decode_bytes(seq_lens, Hq, Hkv, D, max_pages, kv_elem_bytes=2):
     """Algorithmic bytes: every cached K and V row once, plus q, o, lse, tables."""
     toks = int(sum(seq_lens))
     n = len(seq_lens)
-    kv = toks * Hkv * D * 2 * 2
+    kv = toks * Hkv * D * kv_elem_bytes * 2
     return kv + n * Hq * D * 2 * 2 + n * Hq * 4 + n * max_pages * 4 + n * 4
 
 
@@ -367,12 +367,55 @@ def run_gpu(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_blasst:
         line["blasst_long_context"] = blasst_long_context_report(dev)
         line["chunked_prefill_paged"] = chunked_prefill_report(dev, peaks)
+        line["decode_fp8"] = fp8_decode_report(dev, peaks, cache, flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfs, gbs, secs, desc = oracle_sample(int(args.cpu_heads), 4)
         line["cpu_baseline"] = {"value": tfs, "unit": "TFLOP/s", "cores": cpu_threads()[0], "kind": "oracle",
                                 "sample": desc, "decode_gbs": gbs, "seconds": secs}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def fp8_decode_report(dev, peaks, cache, flush, reps=10):
+    """The decode workload above with its page pools stored as FP8 E4M3 codes
+    (one scale per pool): same sequences, split and query; half the cache bytes."""
+    import attention_online_softmax_fwd_b200 as ab
+    dc = gen.CONFIGS[DECODE_CFG]
+    kc, ks = gen.quantize_pool_e4m3(cache.k_pages)
+    vc, vs = gen.quantize_pool_e4m3(cache.v_pages)
+    args = [t.to(dev) for t in (cache.q, kc, vc)]
+    bt, sl = cache.block_table.to(dev), cache.seq_lens.to(dev)
+    o = torch.empty_like(args[0])
+    lse = torch.empty((dc["N"], dc["Hq"]), dtype=torch.float32, device=dev)
+    ws = torch.empty(ab.decode_workspace_bytes(dc["N"], dc["Hq"], dc["D"], cache.max_pages, dc["page_size"],
+                                               DECODE_SPLIT), dtype=torch.uint8, device=dev)
+    scale = gen.attn_scale(dc["D"])
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        ab.decode_paged_fp8(args[0], args[1], args[2], ks, vs, bt, sl, scale=scale, split_tokens=DECODE_SPLIT,
+                            out=o, lse=lse, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.mean(ts)
+    by = decode_bytes(cache.seq_lens.tolist(), dc["Hq"], dc["Hkv"], dc["D"], cache.max_pages, kv_elem_bytes=1)
+    gbs = by / (ms * 1e-3) / 1e9
+    return {"workload": f"{DECODE_CFG} with E4M3 K/V pools, split {DECODE_SPLIT}",
+            "kernel": "decode_heads_kernel<128,4,8,fp8>+decode_merge_kernel", "ms": ms, "gbs": gbs,
+            "bytes_per_call": by, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
+            "frac_of_spec_8000": gbs / SPEC_PEAKS["hbm_gbs"],
+            "tokens_per_s": int(cache.seq_lens.sum()) / (ms * 1e-3)}
 
 
 def chunked_prefill_report(dev, peaks, reps=5):

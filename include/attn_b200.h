@@ -229,6 +229,32 @@ int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const voi
                                    uint8_t* skip_mask, int* device_status, void* stream);
 
 /*
+ * attn_decode_paged_fp8 -- attn_decode_paged (dense) over a cache stored as
+ * FP8 E4M3 codes. The TensorRT-LLM page ("TensorRT-LLM：大模型推理优化利器",
+ * section 量化) names FP8 among the low-precision formats that cut memory and
+ * bandwidth, and the integration page ("flash-attention与TensorRT-LLM集成")
+ * stores in FP8; neither fixes how the codes are scaled. Reading taken: one
+ * scale per pool, K = k_scale * e4m3(code), V = v_scale * e4m3(code), where
+ * e4m3 is the 1-4-3 format with exponent bias 7, subnormals at exponent 0, no
+ * infinities and S.1111.111 as NaN (largest finite value 448).
+ *   k_codes, v_codes [num_pages][page_size][Hkv][D] uint8 device codes
+ *   k_scale, v_scale finite, > 0
+ * Every other argument, the layouts, the workspace (attn_decode_workspace_bytes
+ * with the same sizes), the results and the errors are those of
+ * attn_decode_paged with lambda = 0 and skip_mask = NULL. Supported: D = 128;
+ * Hkv = 4 or a multiple of 8; Hq / Hkv in {1, 2, 4, 8, 16}; otherwise
+ * ATTN_ERR_UNSUPPORTED. The query stays bf16 and is widened to f16 in the
+ * kernel, so |q| must stay inside the f16 range (65504).
+ */
+int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_codes,
+                          float k_scale, float v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens,
+                          int num_seqs, int Hq, int Hkv, int D, int page_size,
+                          int max_pages_per_seq, int num_pages, float scale, int split_tokens,
+                          void* o, float* lse, void* workspace, size_t workspace_bytes,
+                          int* device_status, void* stream);
+
+/*
  * attn_decode_paged_noalloc -- attn_decode_paged without a caller-provided
  * workspace. (Library plumbing: the pages describe no counterpart.)
  *

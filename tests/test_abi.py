@@ -161,3 +161,33 @@ def test_kv_append_rejects_bad_arguments(lib, bad):
 
 def test_kv_append_rejects_unsupported_head_dim(lib):
     assert _append(lib, D=80) == UNSUPPORTED
+
+
+def _decode_fp8(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, ks=0.01, vs=0.02, bt=FAKE, sl=FAKE, N=4, Hq=32, Hkv=8, D=128, ps=16, mp=8,
+             P=64, scale=0.09, split=64, o=FAKE, lse=None, ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    return lib.attn_decode_paged_fp8(a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["bt"], a["sl"], a["N"],
+                                     a["Hq"], a["Hkv"], a["D"], a["ps"], a["mp"], a["P"], a["scale"], a["split"],
+                                     a["o"], a["lse"], a["ws"], a["wsb"], None, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(kc=None), dict(vc=None), dict(bt=None), dict(sl=None),
+                                 dict(ws=None), dict(o=None), dict(N=0), dict(Hq=12, Hkv=8), dict(ps=24),
+                                 dict(split=96), dict(mp=0), dict(P=0), dict(wsb=16), dict(ks=0.0),
+                                 dict(vs=-1.0), dict(ks=float("nan")), dict(vs=float("inf")), dict(scale=0.0),
+                                 dict(kc=ctypes.c_void_p((1 << 20) + 4)), dict(bt=ctypes.c_void_p((1 << 20) + 2))])
+def test_decode_fp8_rejects_bad_arguments(lib, bad):
+    assert _decode_fp8(lib, **bad) == INVALID
+
+
+@pytest.mark.parametrize("bad", [dict(D=64), dict(Hq=4, Hkv=2), dict(Hq=12, Hkv=12), dict(Hq=64, Hkv=2)])
+def test_decode_fp8_rejects_unsupported(lib, bad):
+    assert _decode_fp8(lib, **bad) == UNSUPPORTED
+
+
+def test_decode_fp8_valid_arguments_without_a_device_report_cuda_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert _decode_fp8(lib) == CUDA
