@@ -236,30 +236,45 @@ int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
-  const long long grid = items < sms ? items : sms;
+  const long long slots = (long long)sms * DecodeHeadsSmem<D, G, HG, F8>::kBlocks;
+  const long long grid = items < slots ? items : slots;
   kernel<<<dim3(unsigned(grid)), dim3((HG + 1) * 32), smem, stream>>>(tk, tv, p, ticket_counter);
   if (int st = launch_status()) return st;
   return launch_merge<D>(p, stream);
 }
 
-template <int D, int HG, bool F8 = false>
+template <int D, int HG>
 int dispatch_decode_heads_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int* ctr,
                             int sms, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_decode_heads<D, 1, HG, F8>(tk, tv, p, ctr, sms, s);
-    case 2: return launch_decode_heads<D, 2, HG, F8>(tk, tv, p, ctr, sms, s);
-    case 4: return launch_decode_heads<D, 4, HG, F8>(tk, tv, p, ctr, sms, s);
-    case 8: return launch_decode_heads<D, 8, HG, F8>(tk, tv, p, ctr, sms, s);
-    case 16: return launch_decode_heads<D, 16, HG, F8>(tk, tv, p, ctr, sms, s);
+    case 1: return launch_decode_heads<D, 1, HG>(tk, tv, p, ctr, sms, s);
+    case 2: return launch_decode_heads<D, 2, HG>(tk, tv, p, ctr, sms, s);
+    case 4: return launch_decode_heads<D, 4, HG>(tk, tv, p, ctr, sms, s);
+    case 8: return launch_decode_heads<D, 8, HG>(tk, tv, p, ctr, sms, s);
+    case 16: return launch_decode_heads<D, 16, HG>(tk, tv, p, ctr, sms, s);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
 
-template <int D, bool F8 = false>
+template <int D>
 int dispatch_decode_heads(int G, int hg, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           int* ctr, int sms, cudaStream_t s) {
-  return hg == 8 ? dispatch_decode_heads_g<D, 8, F8>(G, tk, tv, p, ctr, sms, s)
-                 : dispatch_decode_heads_g<D, 4, F8>(G, tk, tv, p, ctr, sms, s);
+  return hg == 8 ? dispatch_decode_heads_g<D, 8>(G, tk, tv, p, ctr, sms, s)
+                 : dispatch_decode_heads_g<D, 4>(G, tk, tv, p, ctr, sms, s);
+}
+
+// FP8 cache (D = 128): groups of 4 KV heads for G <= 8; G = 16 takes groups of hg (8 or 4)
+int dispatch_decode_heads_fp8(int G, int hg, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                              int* ctr, int sms, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_decode_heads<128, 1, 4, true>(tk, tv, p, ctr, sms, s);
+    case 2: return launch_decode_heads<128, 2, 4, true>(tk, tv, p, ctr, sms, s);
+    case 4: return launch_decode_heads<128, 4, 4, true>(tk, tv, p, ctr, sms, s);
+    case 8: return launch_decode_heads<128, 8, 4, true>(tk, tv, p, ctr, sms, s);
+    case 16: return hg == 8 ? launch_decode_heads<128, 16, 8, true>(tk, tv, p, ctr, sms, s)
+                            : launch_decode_heads<128, 16, 4, true>(tk, tv, p, ctr, sms, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace
@@ -497,7 +512,8 @@ int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_code
   if (D != 128) return ATTN_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return ATTN_ERR_UNSUPPORTED;
-  const int hg = Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0);
+  // G <= 8: groups of 4 KV heads (several CTAs per SM); G = 16: groups of 8 (or all 4)
+  const int hg = G <= 8 ? (Hkv % 4 == 0 ? 4 : 0) : (Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0));
   if (hg == 0) return ATTN_ERR_UNSUPPORTED;
   const size_t need = attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens);
   if (need == 0 || workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
@@ -543,7 +559,7 @@ int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_code
     return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ticket_counter, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
-  return dispatch_decode_heads<128, true>(G, hg, hk, hv, p, ticket_counter, sms, s);
+  return dispatch_decode_heads_fp8(G, hg, hk, hv, p, ticket_counter, sms, s);
 }
 
 }  // extern "C"

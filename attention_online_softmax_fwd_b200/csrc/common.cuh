@@ -300,6 +300,14 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t& lo, u
       : "=r"(lo), "=r"(hi)
       : "r"(four));
 }
+// Transpose of an 8x8 matrix of 16-bit values held one row pair per lane
+// (lane 4r + c holds row r, columns 2c and 2c + 1): returns the same slot of
+// the transposed matrix.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
 // A bf16 pair -> f16 pair (exact inside the f16 range).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));

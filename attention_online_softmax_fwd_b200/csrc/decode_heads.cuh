@@ -37,15 +37,25 @@
 
 namespace attn {
 
-constexpr int kDhChunk = 16;  // tokens per stage
+constexpr int kDhChunk = 16;  // tokens per TMA copy (one 16-slot block of a page)
+
+// The FP8 path for G <= 8 runs 32-token stages (two copies per tensor), several
+// CTAs per SM and fewer stages each: with 4 KV heads per CTA that keeps three
+// 5-warp CTAs resident, so more consumer warps hide each other's latency.
+constexpr int kF8Blocks = 3;   // resident CTAs per SM for G <= 4 (registers: 3 x 160 threads x <= 136)
 
 template <int D, int G, int HG, bool F8 = false>
 struct DecodeHeadsSmem {
+  static constexpr bool kWide = F8 && G <= 8;                    // 32-token stages
+  static constexpr int kHalves = kWide ? 2 : 1;                  // 16-token copies per tensor per stage
+  static constexpr int kTok = kDhChunk * kHalves;                // tokens per stage
+  static constexpr int kBlocks = kWide ? (G <= 4 ? kF8Blocks : 2) : 1;   // resident CTAs per SM
   static constexpr int kHeadBytes = kDhChunk * D * (F8 ? 1 : 2);   // one head's 16 tokens
-  static constexpr int kKVBytes = HG * kHeadBytes;      // K (or V) rows of one stage
+  static constexpr int kHalfBytes = HG * kHeadBytes;             // one copy: 16 tokens of the HG heads
+  static constexpr int kKVBytes = kHalves * kHalfBytes;          // K (or V) rows of one stage
   static constexpr int kQBytes = HG * G * D * 2;        // the item's query rows
   static constexpr int kStageBytes = (2 * kKVBytes + kQBytes + 1023) / 1024 * 1024;
-  static constexpr int kFit = (232448 - 2048) / (kStageBytes + 48);
+  static constexpr int kFit = (233472 / kBlocks - 1024 - 2048) / (kStageBytes + 48);
   static constexpr int kStages = kFit < 8 ? kFit : 8;
   static constexpr int kRing = kStages * kStageBytes;
   static constexpr int kFull = kRing;
@@ -68,7 +78,7 @@ __device__ __forceinline__ void dh_item_coords(long long item, int num_seqs, int
 }
 
 template <int D, int G, int HG, bool F8 = false>
-__global__ void __launch_bounds__((HG + 1) * 32, 1)
+__global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::kBlocks)
     decode_heads_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeParams p, int* ticket_counter) {
   static_assert(G >= 1 && G <= 16, "query heads per KV head");
@@ -151,38 +161,56 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         win_next = e < p.max_pages ? __ldg(&bt_row[e]) : -1;
       }
       const __nv_bfloat16* qsrc = p.q + (size_t(seq) * p.Hq + size_t(grp) * HG * G) * D;
-      for (int t0 = t_begin; t0 < t_end && ok; t0 += kDhChunk) {
+      for (int t0 = t_begin; t0 < t_end && ok; t0 += L::kTok) {
         const int e0 = t0 / p.page_size;
-        if ((e0 >> 5) != win) {
+        if ((e0 >> 5) != win) {   // a stage advances by at most two pages, so by at most one window
           win = e0 >> 5;
           win_cur = win_next;
           const int e = (win + 1) * 32 + lane;
           win_next = e < p.max_pages ? __ldg(&bt_row[e]) : -1;
         }
         if (!mbar_wait(&empty[slot], phase ^ 1u, &abort_flag, p.status)) { ok = false; break; }
-        const int page = __shfl_sync(0xffffffffu, win_cur, e0 & 31);
+        // the page of each 16-token copy (the second may sit on the next page, even in the next window)
+        int page[L::kHalves];
+#pragma unroll
+        for (int h = 0; h < L::kHalves; ++h) {
+          const int e = (t0 + h * kDhChunk) / p.page_size;
+          page[h] = __shfl_sync(0xffffffffu, (e >> 5) == win ? win_cur : win_next, e & 31);
+        }
         if (lane == 0) {
-          const bool valid = page >= 0 && page < p.num_pages;
-          if (!valid) raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
           const bool first = t0 == t_begin;
           TileInfo ti;
           ti.seq = seq; ti.split = split; ti.kvh = grp; ti.t0 = t0;
-          ti.ntok = min(kDhChunk, len - t0);
-          ti.bad = valid ? 0 : 1;
-          ti.flags = (first ? 1 : 0) | (t0 + kDhChunk >= t_end ? 2 : 0);
+          ti.ntok = min(L::kTok, len - t0);
+          ti.bad = 0;
+          uint32_t bytes = first ? uint32_t(L::kQBytes) : 0u;
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h) {
+            if (h * kDhChunk >= ti.ntok) { ti.bad |= 1 << h; continue; }   // past the end: not copied
+            if (page[h] >= 0 && page[h] < p.num_pages) {
+              bytes += uint32_t(2 * L::kHalfBytes);
+            } else {
+              raise_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
+              ti.bad |= 1 << h;
+            }
+          }
+          ti.flags = (first ? 1 : 0) | (t0 + L::kTok >= t_end ? 2 : 0);
           ti.len = len;
           info[slot] = ti;
           uint8_t* stage = smem + slot * L::kStageBytes;
-          mbar_arrive_expect_tx(&full[slot], (valid ? uint32_t(2 * L::kKVBytes) : 0u) + (first ? uint32_t(L::kQBytes) : 0u));
+          mbar_arrive_expect_tx(&full[slot], bytes);
           if (first) bulk_load(stage + 2 * L::kKVBytes, qsrc, uint32_t(L::kQBytes), &full[slot]);
-          if (valid) {
-            const int in_page = t0 % p.page_size;
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h) {
+            if (ti.bad & (1 << h)) continue;
+            const int in_page = (t0 + h * kDhChunk) % p.page_size;
+            uint8_t* kdst = stage + h * L::kHalfBytes;
             if constexpr (F8) {
-              tma_load_4d(stage, &tm_k, &full[slot], 0, in_page, grp * HG, page);
-              tma_load_4d(stage + L::kKVBytes, &tm_v, &full[slot], 0, in_page, grp * HG, page);
+              tma_load_4d(kdst, &tm_k, &full[slot], 0, in_page, grp * HG, page[h]);
+              tma_load_4d(kdst + L::kKVBytes, &tm_v, &full[slot], 0, in_page, grp * HG, page[h]);
             } else {
-              tma_load_5d(stage, &tm_k, &full[slot], 0, 0, in_page, grp * HG, page);
-              tma_load_5d(stage + L::kKVBytes, &tm_v, &full[slot], 0, 0, in_page, grp * HG, page);
+              tma_load_5d(kdst, &tm_k, &full[slot], 0, 0, in_page, grp * HG, page[h]);
+              tma_load_5d(kdst + L::kKVBytes, &tm_v, &full[slot], 0, 0, in_page, grp * HG, page[h]);
             }
           }
         }
@@ -206,6 +234,210 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     if (!ok && lane == 0) {
       for (int s = 0; s < NS; ++s)
         if (pending & (1u << s)) mbar_drain(&full[s], (pending_phase >> s) & 1u);
+    }
+  } else if constexpr (L::kWide) {
+    // ------------------------------------------------------------ consumer warp, FP8 cache, G <= 8: transposed
+    // S^T = K q^T (tokens on the 16-row side, query heads on the 8 columns) and O^T = V^T P^T, so that
+    // one mma covers 16 tokens x G heads: half the mma, exp2 and accumulator count of the untransposed
+    // form. Lane (g, t): S^T rows (tokens) g and g + 8, columns (heads) 2t and 2t + 1; the m-tile m of
+    // O^T has rows = head dims 16r + m (r < 8) and 16(r - 8) + 8 + m (r >= 8), so lane (g, t) ends up
+    // with dims 16g .. 16g + 15 of heads 2t and 2t + 1. P^T goes from the S^T accumulator layout to the
+    // P^T operand layout with one 8x8 transpose per 8 tokens.
+    const float neg_inf = -__int_as_float(0x7f800000);
+    const int g = lane >> 2, tq = lane & 3;
+    const bool head_valid[2] = {2 * tq < G, 2 * tq + 1 < G};
+    int slot = 0;
+    uint32_t phase = 0;
+    int no_abort = 0;
+    bool ok = true;
+    int seq = 0, split = 0, grp = 0, n_splits = 0;
+    uint32_t qb[KS][2];
+    float o[8][4];
+    float m_ref[2] = {neg_inf, neg_inf};   // heads 2tq, 2tq + 1
+    float l_part[2] = {0.f, 0.f};
+    float lr_part[2] = {0.f, 0.f};
+
+    while (ok) {
+      if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) { ok = false; break; }
+      const TileInfo ti = info[slot];
+      if (ti.flags & 4) break;
+      uint8_t* stage = smem + slot * L::kStageBytes;
+      if (ti.flags & 1) {
+        seq = ti.seq; split = ti.split; grp = ti.kvh;
+        n_splits = (ti.len + p.split_tokens - 1) / p.split_tokens;
+        // q^T operand: column g = query head g of this KV head, dims 32tq + 4ks + {0,1} / {2,3}
+        const uint32_t* qs = reinterpret_cast<const uint32_t*>(stage + 2 * L::kKVBytes) + warp * G * (D / 2);
+        const bool qv = g < G;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qb[ks][0] = qv ? bf16x2_to_f16x2(qs[g * (D / 2) + 16 * tq + 2 * ks]) : 0u;
+          qb[ks][1] = qv ? bf16x2_to_f16x2(qs[g * (D / 2) + 16 * tq + 2 * ks + 1]) : 0u;
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+        m_ref[0] = m_ref[1] = neg_inf;
+        l_part[0] = l_part[1] = 0.f;
+        lr_part[0] = lr_part[1] = 0.f;
+      }
+      const bool last = (ti.flags & 2) != 0;
+      if (ti.bad != (1 << L::kHalves) - 1) {
+        const int ntok = ti.ntok;
+        const int bad = ti.bad;
+        // ---- S^T = K q^T per 16-token half: key rows g and g + 8 (swizzle phase g), bytes [32tq, 32tq + 32)
+        float st[L::kHalves][4];
+#pragma unroll
+        for (int h = 0; h < L::kHalves; ++h) {
+          float sp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          const uint8_t* kb = stage + h * L::kHalfBytes + warp * L::kHeadBytes;
+          const uint4 r0a = *reinterpret_cast<const uint4*>(kb + g * 128 + (((2 * tq) ^ g) << 4));
+          const uint4 r0b = *reinterpret_cast<const uint4*>(kb + g * 128 + (((2 * tq + 1) ^ g) << 4));
+          const uint4 r1a = *reinterpret_cast<const uint4*>(kb + (g + 8) * 128 + (((2 * tq) ^ g) << 4));
+          const uint4 r1b = *reinterpret_cast<const uint4*>(kb + (g + 8) * 128 + (((2 * tq + 1) ^ g) << 4));
+          const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
+          const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4];
+            e4m3x4_to_f16x2x2(w0[ks], a[0], a[2]);
+            e4m3x4_to_f16x2x2(w1[ks], a[1], a[3]);
+            mma_f16_16816(sp[ks & 1], a, qb[ks][0], qb[ks][1]);
+          }
+          // st[h][e]: token 16h + g + 8 (e >> 1), head 2tq + (e & 1); half h not copied -> all masked
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tok = h * kDhChunk + g + 8 * (e >> 1);
+            const float v = (sp[0][e] + sp[1][e]) * p.scale_log2;
+            st[h][e] = (!head_valid[e & 1] || tok >= ntok || ((bad >> h) & 1)) ? neg_inf : v;
+          }
+        }
+        float mx[2] = {fmaxf(st[0][0], st[0][2]), fmaxf(st[0][1], st[0][3])};
+#pragma unroll
+        for (int h = 1; h < L::kHalves; ++h) {
+          mx[0] = fmaxf(mx[0], fmaxf(st[h][0], st[h][2]));
+          mx[1] = fmaxf(mx[1], fmaxf(st[h][1], st[h][3]));
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          mx[c] = fmaxf(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], 4));
+          mx[c] = fmaxf(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], 8));
+          mx[c] = fmaxf(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], 16));
+        }
+        float alpha[2] = {1.f, 1.f};
+        bool raised = false;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (mx[c] != neg_inf && (m_ref[c] == neg_inf || mx[c] > m_ref[c] + kDecRescaleThreshold)) {
+            alpha[c] = (m_ref[c] == neg_inf) ? 0.f : fast_exp2(m_ref[c] - mx[c]);
+            m_ref[c] = mx[c];
+            raised = true;
+          }
+        }
+        if (__any_sync(0xffffffffu, raised)) {
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            o[m][0] *= alpha[0]; o[m][2] *= alpha[0];
+            o[m][1] *= alpha[1]; o[m][3] *= alpha[1];
+          }
+          l_part[0] *= alpha[0]; lr_part[0] *= alpha[0];
+          l_part[1] *= alpha[1]; lr_part[1] *= alpha[1];
+        }
+        uint32_t pb[L::kHalves][2];   // P^T operand per half: tokens 2tq, 2tq + 1 (and + 8) of head g
+        {
+          const float off[2] = {m_ref[0] == neg_inf ? 0.f : m_ref[0], m_ref[1] == neg_inf ? 0.f : m_ref[1]};
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h) {
+            float pr[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(st[h][e] - off[e & 1]);
+            const uint32_t x0 = pack_f16x2(pr[0], pr[1]);   // token g, heads 2tq, 2tq + 1
+            const uint32_t x1 = pack_f16x2(pr[2], pr[3]);   // token g + 8
+            l_part[0] += pr[0] + pr[2];
+            l_part[1] += pr[1] + pr[3];
+            // the weights applied to V are normalised by the sum of the rounded P
+            lr_part[0] += f16_lo(x0) + f16_lo(x1);
+            lr_part[1] += f16_hi(x0) + f16_hi(x1);
+            pb[h][0] = movmatrix_trans(x0);
+            pb[h][1] = movmatrix_trans(x1);
+          }
+        }
+        // ---- O^T += V^T P^T per half: token rows 2tq, 2tq + 1, 2tq + 8, 2tq + 9, byte group g (dims 16g ..);
+        // rows past the end or of a half not copied are zeroed so that 0 * (stale or NaN) cannot reach O
+#pragma unroll
+        for (int h = 0; h < L::kHalves; ++h) {
+          if ((bad >> h) & 1) continue;
+          const uint8_t* vb = stage + L::kKVBytes + h * L::kHalfBytes + warp * L::kHeadBytes;
+          uint4 vr[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tok = 2 * tq + (i & 1) + (i >> 1) * 8;
+            vr[i] = *reinterpret_cast<const uint4*>(vb + tok * 128 + ((g ^ (tok & 7)) << 4));
+            if (h * kDhChunk + tok >= ntok) vr[i] = make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            // m-tiles 4w .. 4w + 3: rows g (dim 16g + m, word w) and g + 8 (dim 16g + 8 + m, word w + 2)
+            uint32_t a0[4], a1[4], a2[4], a3[4];
+            const uint32_t A0 = (&vr[0].x)[w], B0 = (&vr[1].x)[w], C0 = (&vr[2].x)[w], D0 = (&vr[3].x)[w];
+            const uint32_t A1 = (&vr[0].x)[w + 2], B1 = (&vr[1].x)[w + 2], C1 = (&vr[2].x)[w + 2],
+                           D1 = (&vr[3].x)[w + 2];
+            e4m3x4_to_f16x2x2(__byte_perm(A0, B0, 0x5140), a0[0], a0[1]);
+            e4m3x4_to_f16x2x2(__byte_perm(A0, B0, 0x7362), a0[2], a0[3]);
+            e4m3x4_to_f16x2x2(__byte_perm(A1, B1, 0x5140), a1[0], a1[1]);
+            e4m3x4_to_f16x2x2(__byte_perm(A1, B1, 0x7362), a1[2], a1[3]);
+            e4m3x4_to_f16x2x2(__byte_perm(C0, D0, 0x5140), a2[0], a2[1]);
+            e4m3x4_to_f16x2x2(__byte_perm(C0, D0, 0x7362), a2[2], a2[3]);
+            e4m3x4_to_f16x2x2(__byte_perm(C1, D1, 0x5140), a3[0], a3[1]);
+            e4m3x4_to_f16x2x2(__byte_perm(C1, D1, 0x7362), a3[2], a3[3]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t a[4] = {a0[i], a1[i], a2[i], a3[i]};
+              mma_f16_16816(o[4 * w + i], a, pb[h][0], pb[h][1]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (++slot == NS) { slot = 0; phase ^= 1u; }
+      if (!last) continue;
+
+      // ---- the item's result for heads 2tq, 2tq + 1 of this warp's KV head
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        l_part[c] += __shfl_xor_sync(0xffffffffu, l_part[c], 4);
+        l_part[c] += __shfl_xor_sync(0xffffffffu, l_part[c], 8);
+        l_part[c] += __shfl_xor_sync(0xffffffffu, l_part[c], 16);
+        lr_part[c] += __shfl_xor_sync(0xffffffffu, lr_part[c], 4);
+        lr_part[c] += __shfl_xor_sync(0xffffffffu, lr_part[c], 8);
+        lr_part[c] += __shfl_xor_sync(0xffffffffu, lr_part[c], 16);
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (!head_valid[c]) continue;
+        const int hq = (grp * HG + warp) * G + 2 * tq + c;
+        const float lsum = l_part[c];
+        const float inv = (lr_part[c] > 0.f ? 1.f / lr_part[c] : 0.f) * p.v_scale;
+        if (n_splits == 1) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(seq) * p.Hq + hq) * D + 16 * g);
+          dst[0] = make_uint4(pack_bf16x2(o[0][c] * inv, o[1][c] * inv), pack_bf16x2(o[2][c] * inv, o[3][c] * inv),
+                              pack_bf16x2(o[4][c] * inv, o[5][c] * inv), pack_bf16x2(o[6][c] * inv, o[7][c] * inv));
+          dst[1] = make_uint4(pack_bf16x2(o[0][c + 2] * inv, o[1][c + 2] * inv),
+                              pack_bf16x2(o[2][c + 2] * inv, o[3][c + 2] * inv),
+                              pack_bf16x2(o[4][c + 2] * inv, o[5][c + 2] * inv),
+                              pack_bf16x2(o[6][c + 2] * inv, o[7][c + 2] * inv));
+          if (p.lse && g == 0)
+            p.lse[size_t(seq) * p.Hq + hq] = lsum > 0.f ? (m_ref[c] + __log2f(lsum)) * 0.69314718055994531f : neg_inf;
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D +
+                                                  16 * g);
+          dst[0] = make_float4(o[0][c] * inv, o[1][c] * inv, o[2][c] * inv, o[3][c] * inv);
+          dst[1] = make_float4(o[4][c] * inv, o[5][c] * inv, o[6][c] * inv, o[7][c] * inv);
+          dst[2] = make_float4(o[0][c + 2] * inv, o[1][c + 2] * inv, o[2][c + 2] * inv, o[3][c + 2] * inv);
+          dst[3] = make_float4(o[4][c + 2] * inv, o[5][c + 2] * inv, o[6][c + 2] * inv, o[7][c + 2] * inv);
+          if (g == 0)
+            p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lsum > 0.f ? m_ref[c] + __log2f(lsum) : neg_inf;
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ consumer warp = KV head `warp` of the group

@@ -242,7 +242,8 @@ int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const voi
  * Every other argument, the layouts, the workspace (attn_decode_workspace_bytes
  * with the same sizes), the results and the errors are those of
  * attn_decode_paged with lambda = 0 and skip_mask = NULL. Supported: D = 128;
- * Hkv = 4 or a multiple of 8; Hq / Hkv in {1, 2, 4, 8, 16}; otherwise
+ * Hkv a multiple of 4 (Hq / Hkv = 16: Hkv = 4 or a multiple of 8);
+ * Hq / Hkv in {1, 2, 4, 8, 16}; otherwise
  * ATTN_ERR_UNSUPPORTED. The query stays bf16 and is widened to f16 in the
  * kernel, so |q| must stay inside the f16 range (65504).
  */

@@ -181,7 +181,7 @@ def test_decode_fp8_rejects_bad_arguments(lib, bad):
     assert _decode_fp8(lib, **bad) == INVALID
 
 
-@pytest.mark.parametrize("bad", [dict(D=64), dict(Hq=4, Hkv=2), dict(Hq=12, Hkv=12), dict(Hq=64, Hkv=2)])
+@pytest.mark.parametrize("bad", [dict(D=64), dict(Hq=4, Hkv=2), dict(Hq=12, Hkv=6), dict(Hq=64, Hkv=2), dict(Hq=192, Hkv=12)])
 def test_decode_fp8_rejects_unsupported(lib, bad):
     assert _decode_fp8(lib, **bad) == UNSUPPORTED
 
