@@ -243,24 +243,19 @@ int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
   return launch_merge<D>(p, stream);
 }
 
-template <int D, int HG>
-int dispatch_decode_heads_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int* ctr,
-                            int sms, cudaStream_t s) {
-  switch (G) {
-    case 1: return launch_decode_heads<D, 1, HG>(tk, tv, p, ctr, sms, s);
-    case 2: return launch_decode_heads<D, 2, HG>(tk, tv, p, ctr, sms, s);
-    case 4: return launch_decode_heads<D, 4, HG>(tk, tv, p, ctr, sms, s);
-    case 8: return launch_decode_heads<D, 8, HG>(tk, tv, p, ctr, sms, s);
-    case 16: return launch_decode_heads<D, 16, HG>(tk, tv, p, ctr, sms, s);
-    default: return ATTN_ERR_UNSUPPORTED;
-  }
-}
-
+// groups of 4 KV heads for G <= 8 (several CTAs per SM); G = 16 takes groups of hg (8 or 4)
 template <int D>
 int dispatch_decode_heads(int G, int hg, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           int* ctr, int sms, cudaStream_t s) {
-  return hg == 8 ? dispatch_decode_heads_g<D, 8>(G, tk, tv, p, ctr, sms, s)
-                 : dispatch_decode_heads_g<D, 4>(G, tk, tv, p, ctr, sms, s);
+  switch (G) {
+    case 1: return launch_decode_heads<D, 1, 4>(tk, tv, p, ctr, sms, s);
+    case 2: return launch_decode_heads<D, 2, 4>(tk, tv, p, ctr, sms, s);
+    case 4: return launch_decode_heads<D, 4, 4>(tk, tv, p, ctr, sms, s);
+    case 8: return launch_decode_heads<D, 8, 4>(tk, tv, p, ctr, sms, s);
+    case 16: return hg == 8 ? launch_decode_heads<D, 16, 8>(tk, tv, p, ctr, sms, s)
+                            : launch_decode_heads<D, 16, 4>(tk, tv, p, ctr, sms, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
 }
 
 // FP8 cache (D = 128): groups of 4 KV heads for G <= 8; G = 16 takes groups of hg (8 or 4)
@@ -421,7 +416,7 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
   if (int st = encode_map5(&tv, v_pages, dims, strides, box)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool use_skip = lambda > 0.f || skip_mask != nullptr || per_head;
-  const int hg = Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0);
+  const int hg = G <= 8 ? (Hkv % 4 == 0 ? 4 : 0) : (Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0));
   if (!use_skip && hg > 0) {
     // dense: one item per group of hg KV heads, 16-token stages covering all of them
     const uint64_t hdims[5] = {64, uint64_t(D / 64), uint64_t(page_size), uint64_t(Hkv), uint64_t(num_pages)};

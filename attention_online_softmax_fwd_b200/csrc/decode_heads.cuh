@@ -39,17 +39,19 @@ namespace attn {
 
 constexpr int kDhChunk = 16;  // tokens per TMA copy (one 16-slot block of a page)
 
-// The FP8 path for G <= 8 runs 32-token stages (two copies per tensor), several
-// CTAs per SM and fewer stages each: with 4 KV heads per CTA that keeps three
-// 5-warp CTAs resident, so more consumer warps hide each other's latency.
-constexpr int kF8Blocks = 3;   // resident CTAs per SM for G <= 4 (registers: 3 x 160 threads x <= 136)
+// For G <= 8 the consumers run the transposed products (below) with groups of
+// 4 KV heads and several CTAs per SM, fewer stages each: three 5-warp CTAs
+// (two for G = 8) keep 12 consumer warps resident, which hide each other's
+// latency. The FP8 cache also doubles the stage to 32 tokens (two copies per
+// tensor) to spread the per-stage costs over more tokens.
+constexpr int kTrBlocks = 3;   // resident CTAs per SM for G <= 4 (registers: 3 x 160 threads x <= 136)
 
 template <int D, int G, int HG, bool F8 = false>
 struct DecodeHeadsSmem {
-  static constexpr bool kWide = F8 && G <= 8;                    // 32-token stages
-  static constexpr int kHalves = kWide ? 2 : 1;                  // 16-token copies per tensor per stage
+  static constexpr bool kTr = G <= 8;                            // transposed products
+  static constexpr int kHalves = (kTr && F8) ? 2 : 1;            // 16-token copies per tensor per stage
   static constexpr int kTok = kDhChunk * kHalves;                // tokens per stage
-  static constexpr int kBlocks = kWide ? (G <= 4 ? kF8Blocks : 2) : 1;   // resident CTAs per SM
+  static constexpr int kBlocks = kTr ? (G <= 4 ? kTrBlocks : 2) : 1;   // resident CTAs per SM
   static constexpr int kHeadBytes = kDhChunk * D * (F8 ? 1 : 2);   // one head's 16 tokens
   static constexpr int kHalfBytes = HG * kHeadBytes;             // one copy: 16 tokens of the HG heads
   static constexpr int kKVBytes = kHalves * kHalfBytes;          // K (or V) rows of one stage
@@ -235,14 +237,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
       for (int s = 0; s < NS; ++s)
         if (pending & (1u << s)) mbar_drain(&full[s], (pending_phase >> s) & 1u);
     }
-  } else if constexpr (L::kWide) {
-    // ------------------------------------------------------------ consumer warp, FP8 cache, G <= 8: transposed
+  } else if constexpr (L::kTr) {
+    // ------------------------------------------------------------ consumer warp, G <= 8: transposed products
     // S^T = K q^T (tokens on the 16-row side, query heads on the 8 columns) and O^T = V^T P^T, so that
-    // one mma covers 16 tokens x G heads: half the mma, exp2 and accumulator count of the untransposed
-    // form. Lane (g, t): S^T rows (tokens) g and g + 8, columns (heads) 2t and 2t + 1; the m-tile m of
-    // O^T has rows = head dims 16r + m (r < 8) and 16(r - 8) + 8 + m (r >= 8), so lane (g, t) ends up
-    // with dims 16g .. 16g + 15 of heads 2t and 2t + 1. P^T goes from the S^T accumulator layout to the
-    // P^T operand layout with one 8x8 transpose per 8 tokens.
+    // one mma covers 16 tokens x G heads: half the mma, exp2 and accumulator count of the q-on-rows
+    // form. Lane (g, t): S^T rows (tokens) g and g + 8, columns (heads) 2t and 2t + 1. P^T goes from
+    // the S^T accumulator layout to the P^T operand layout with one 8x8 transpose per 8 tokens.
+    // O^T m-tile m, row r is head dim 16m + r for bf16 (operands from ldmatrix), and 16r + m (r < 8),
+    // 16(r - 8) + 8 + m (r >= 8) for FP8, where lane (g, t) then holds dims 16g .. 16g + 15.
     const float neg_inf = -__int_as_float(0x7f800000);
     const int g = lane >> 2, tq = lane & 3;
     const bool head_valid[2] = {2 * tq < G, 2 * tq + 1 < G};
@@ -251,8 +253,10 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
     int no_abort = 0;
     bool ok = true;
     int seq = 0, split = 0, grp = 0, n_splits = 0;
+    constexpr int MT = D / 16;   // m-tiles of O^T
     uint32_t qb[KS][2];
-    float o[8][4];
+    float o[MT][4];
+    const uint32_t ring_addr = smem_u32(smem);
     float m_ref[2] = {neg_inf, neg_inf};   // heads 2tq, 2tq + 1
     float l_part[2] = {0.f, 0.f};
     float lr_part[2] = {0.f, 0.f};
@@ -265,16 +269,22 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
       if (ti.flags & 1) {
         seq = ti.seq; split = ti.split; grp = ti.kvh;
         n_splits = (ti.len + p.split_tokens - 1) / p.split_tokens;
-        // q^T operand: column g = query head g of this KV head, dims 32tq + 4ks + {0,1} / {2,3}
+        // q^T operand: column g = query head g of this KV head; FP8: dims 32tq + 4ks + {0,1} / {2,3}
+        // (matching the key fragments), bf16: dims 16ks + 2tq + {0,1} / + 8
         const uint32_t* qs = reinterpret_cast<const uint32_t*>(stage + 2 * L::kKVBytes) + warp * G * (D / 2);
         const bool qv = g < G;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
-          qb[ks][0] = qv ? bf16x2_to_f16x2(qs[g * (D / 2) + 16 * tq + 2 * ks]) : 0u;
-          qb[ks][1] = qv ? bf16x2_to_f16x2(qs[g * (D / 2) + 16 * tq + 2 * ks + 1]) : 0u;
+          if constexpr (F8) {
+            qb[ks][0] = qv ? bf16x2_to_f16x2(qs[g * (D / 2) + 16 * tq + 2 * ks]) : 0u;
+            qb[ks][1] = qv ? bf16x2_to_f16x2(qs[g * (D / 2) + 16 * tq + 2 * ks + 1]) : 0u;
+          } else {
+            qb[ks][0] = qv ? qs[g * (D / 2) + ks * 8 + tq] : 0u;
+            qb[ks][1] = qv ? qs[g * (D / 2) + ks * 8 + 4 + tq] : 0u;
+          }
         }
 #pragma unroll
-        for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+        for (int m = 0; m < MT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
         m_ref[0] = m_ref[1] = neg_inf;
         l_part[0] = l_part[1] = 0.f;
         lr_part[0] = lr_part[1] = 0.f;
@@ -288,19 +298,32 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
 #pragma unroll
         for (int h = 0; h < L::kHalves; ++h) {
           float sp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-          const uint8_t* kb = stage + h * L::kHalfBytes + warp * L::kHeadBytes;
-          const uint4 r0a = *reinterpret_cast<const uint4*>(kb + g * 128 + (((2 * tq) ^ g) << 4));
-          const uint4 r0b = *reinterpret_cast<const uint4*>(kb + g * 128 + (((2 * tq + 1) ^ g) << 4));
-          const uint4 r1a = *reinterpret_cast<const uint4*>(kb + (g + 8) * 128 + (((2 * tq) ^ g) << 4));
-          const uint4 r1b = *reinterpret_cast<const uint4*>(kb + (g + 8) * 128 + (((2 * tq + 1) ^ g) << 4));
-          const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
-          const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
+          if constexpr (F8) {
+            const uint8_t* kb = stage + h * L::kHalfBytes + warp * L::kHeadBytes;
+            const uint4 r0a = *reinterpret_cast<const uint4*>(kb + g * 128 + (((2 * tq) ^ g) << 4));
+            const uint4 r0b = *reinterpret_cast<const uint4*>(kb + g * 128 + (((2 * tq + 1) ^ g) << 4));
+            const uint4 r1a = *reinterpret_cast<const uint4*>(kb + (g + 8) * 128 + (((2 * tq) ^ g) << 4));
+            const uint4 r1b = *reinterpret_cast<const uint4*>(kb + (g + 8) * 128 + (((2 * tq + 1) ^ g) << 4));
+            const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
+            const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            uint32_t a[4];
-            e4m3x4_to_f16x2x2(w0[ks], a[0], a[2]);
-            e4m3x4_to_f16x2x2(w1[ks], a[1], a[3]);
-            mma_f16_16816(sp[ks & 1], a, qb[ks][0], qb[ks][1]);
+            for (int ks = 0; ks < KS; ++ks) {
+              uint32_t a[4];
+              e4m3x4_to_f16x2x2(w0[ks], a[0], a[2]);
+              e4m3x4_to_f16x2x2(w1[ks], a[1], a[3]);
+              mma_f16_16816(sp[ks & 1], a, qb[ks][0], qb[ks][1]);
+            }
+          } else {
+            // K operand by ldmatrix: matrix mi = tokens 8 (mi & 1) .., dims 16ks + 8 (mi >> 1) ..
+            const uint32_t kaddr = ring_addr + slot * L::kStageBytes + h * L::kHalfBytes + warp * L::kHeadBytes;
+            const int mi = lane >> 3, r = lane & 7;
+            const int tok = (mi & 1) * 8 + r;
+            uint32_t af[KS][4];
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks)
+              ldsm_x4(kaddr + swz_off<D>(tok, ks * 2 + (mi >> 1)), af[ks][0], af[ks][1], af[ks][2], af[ks][3]);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) mma_bf16_16816(sp[ks & 1], af[ks], qb[ks][0], qb[ks][1]);
           }
           // st[h][e]: token 16h + g + 8 (e >> 1), head 2tq + (e & 1); half h not copied -> all masked
 #pragma unroll
@@ -334,7 +357,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
         }
         if (__any_sync(0xffffffffu, raised)) {
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
+          for (int m = 0; m < MT; ++m) {
             o[m][0] *= alpha[0]; o[m][2] *= alpha[0];
             o[m][1] *= alpha[1]; o[m][3] *= alpha[1];
           }
@@ -349,22 +372,46 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
             float pr[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(st[h][e] - off[e & 1]);
-            const uint32_t x0 = pack_f16x2(pr[0], pr[1]);   // token g, heads 2tq, 2tq + 1
-            const uint32_t x1 = pack_f16x2(pr[2], pr[3]);   // token g + 8
             l_part[0] += pr[0] + pr[2];
             l_part[1] += pr[1] + pr[3];
             // the weights applied to V are normalised by the sum of the rounded P
-            lr_part[0] += f16_lo(x0) + f16_lo(x1);
-            lr_part[1] += f16_hi(x0) + f16_hi(x1);
+            uint32_t x0, x1;   // tokens g and g + 8, heads 2tq, 2tq + 1
+            if constexpr (F8) {
+              x0 = pack_f16x2(pr[0], pr[1]);
+              x1 = pack_f16x2(pr[2], pr[3]);
+              lr_part[0] += f16_lo(x0) + f16_lo(x1);
+              lr_part[1] += f16_hi(x0) + f16_hi(x1);
+            } else {
+              x0 = pack_bf16x2(pr[0], pr[1]);
+              x1 = pack_bf16x2(pr[2], pr[3]);
+              lr_part[0] += bf16_lo(x0) + bf16_lo(x1);
+              lr_part[1] += bf16_hi(x0) + bf16_hi(x1);
+            }
             pb[h][0] = movmatrix_trans(x0);
             pb[h][1] = movmatrix_trans(x1);
           }
         }
         // ---- O^T += V^T P^T per half: token rows 2tq, 2tq + 1, 2tq + 8, 2tq + 9, byte group g (dims 16g ..);
         // rows past the end or of a half not copied are zeroed so that 0 * (stale or NaN) cannot reach O
+        if constexpr (!F8) {
+          // V^T operand by transposing ldmatrix: matrix mi = tokens 8 (mi >> 1) .., dims 16m + 8 (mi & 1) ..;
+          // a[0], a[1] hold tokens 2tq, 2tq + 1 and a[2], a[3] tokens 2tq + 8, 2tq + 9 (low, high half)
+          const uint32_t vaddr = ring_addr + slot * L::kStageBytes + L::kKVBytes + warp * L::kHeadBytes;
+          const int mi = lane >> 3, r = lane & 7;
+          const int tok = (mi >> 1) * 8 + r;
+          const uint32_t mk0 = (2 * tq < ntok ? 0x0000FFFFu : 0u) | (2 * tq + 1 < ntok ? 0xFFFF0000u : 0u);
+          const uint32_t mk1 = (2 * tq + 8 < ntok ? 0x0000FFFFu : 0u) | (2 * tq + 9 < ntok ? 0xFFFF0000u : 0u);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            uint32_t a[4];
+            ldsm_x4_t(vaddr + swz_off<D>(tok, 2 * m + (mi & 1)), a[0], a[1], a[2], a[3]);
+            a[0] &= mk0; a[1] &= mk0; a[2] &= mk1; a[3] &= mk1;
+            mma_bf16_16816(o[m], a, pb[0][0], pb[0][1]);
+          }
+        }
 #pragma unroll
         for (int h = 0; h < L::kHalves; ++h) {
-          if ((bad >> h) & 1) continue;
+          if (!F8 || ((bad >> h) & 1)) continue;
           const uint8_t* vb = stage + L::kKVBytes + h * L::kHalfBytes + warp * L::kHeadBytes;
           uint4 vr[4];
 #pragma unroll
@@ -416,24 +463,43 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
         if (!head_valid[c]) continue;
         const int hq = (grp * HG + warp) * G + 2 * tq + c;
         const float lsum = l_part[c];
-        const float inv = (lr_part[c] > 0.f ? 1.f / lr_part[c] : 0.f) * p.v_scale;
+        float inv = lr_part[c] > 0.f ? 1.f / lr_part[c] : 0.f;   // 0 only if every page was invalid
+        if constexpr (F8) inv *= p.v_scale;
         if (n_splits == 1) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(seq) * p.Hq + hq) * D + 16 * g);
-          dst[0] = make_uint4(pack_bf16x2(o[0][c] * inv, o[1][c] * inv), pack_bf16x2(o[2][c] * inv, o[3][c] * inv),
-                              pack_bf16x2(o[4][c] * inv, o[5][c] * inv), pack_bf16x2(o[6][c] * inv, o[7][c] * inv));
-          dst[1] = make_uint4(pack_bf16x2(o[0][c + 2] * inv, o[1][c + 2] * inv),
-                              pack_bf16x2(o[2][c + 2] * inv, o[3][c + 2] * inv),
-                              pack_bf16x2(o[4][c + 2] * inv, o[5][c + 2] * inv),
-                              pack_bf16x2(o[6][c + 2] * inv, o[7][c + 2] * inv));
+          if constexpr (F8) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(seq) * p.Hq + hq) * D + 16 * g);
+            dst[0] = make_uint4(pack_bf16x2(o[0][c] * inv, o[1][c] * inv), pack_bf16x2(o[2][c] * inv, o[3][c] * inv),
+                                pack_bf16x2(o[4][c] * inv, o[5][c] * inv), pack_bf16x2(o[6][c] * inv, o[7][c] * inv));
+            dst[1] = make_uint4(pack_bf16x2(o[0][c + 2] * inv, o[1][c + 2] * inv),
+                                pack_bf16x2(o[2][c + 2] * inv, o[3][c + 2] * inv),
+                                pack_bf16x2(o[4][c + 2] * inv, o[5][c + 2] * inv),
+                                pack_bf16x2(o[6][c + 2] * inv, o[7][c + 2] * inv));
+          } else {
+            __nv_bfloat16* dst = p.o + (size_t(seq) * p.Hq + hq) * D + g;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              dst[16 * m] = __float2bfloat16_rn(o[m][c] * inv);
+              dst[16 * m + 8] = __float2bfloat16_rn(o[m][c + 2] * inv);
+            }
+          }
           if (p.lse && g == 0)
             p.lse[size_t(seq) * p.Hq + hq] = lsum > 0.f ? (m_ref[c] + __log2f(lsum)) * 0.69314718055994531f : neg_inf;
         } else {
-          float4* dst = reinterpret_cast<float4*>(p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D +
-                                                  16 * g);
-          dst[0] = make_float4(o[0][c] * inv, o[1][c] * inv, o[2][c] * inv, o[3][c] * inv);
-          dst[1] = make_float4(o[4][c] * inv, o[5][c] * inv, o[6][c] * inv, o[7][c] * inv);
-          dst[2] = make_float4(o[0][c + 2] * inv, o[1][c + 2] * inv, o[2][c + 2] * inv, o[3][c + 2] * inv);
-          dst[3] = make_float4(o[4][c + 2] * inv, o[5][c + 2] * inv, o[6][c + 2] * inv, o[7][c + 2] * inv);
+          if constexpr (F8) {
+            float4* dst = reinterpret_cast<float4*>(p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D +
+                                                    16 * g);
+            dst[0] = make_float4(o[0][c] * inv, o[1][c] * inv, o[2][c] * inv, o[3][c] * inv);
+            dst[1] = make_float4(o[4][c] * inv, o[5][c] * inv, o[6][c] * inv, o[7][c] * inv);
+            dst[2] = make_float4(o[0][c + 2] * inv, o[1][c + 2] * inv, o[2][c + 2] * inv, o[3][c + 2] * inv);
+            dst[3] = make_float4(o[4][c + 2] * inv, o[5][c + 2] * inv, o[6][c + 2] * inv, o[7][c + 2] * inv);
+          } else {
+            float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + g;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              dst[16 * m] = o[m][c] * inv;
+              dst[16 * m + 8] = o[m][c + 2] * inv;
+            }
+          }
           if (g == 0)
             p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lsum > 0.f ? m_ref[c] + __log2f(lsum) : neg_inf;
         }
