@@ -194,11 +194,24 @@ long long max_splits_of(int max_pages, int page_size, int split_tokens) {
   return (cap + split_tokens - 1) / split_tokens;
 }
 
-// One CTA per (sequence, query head); a no-op for sequences of one split.
+// One CTA per (sequence, query head); a no-op for sequences of one split. Launched
+// as a programmatic dependent of the split kernel: it is scheduled while the split
+// kernel's last CTAs run and waits (griddepcontrol.wait) for that grid to finish
+// and its writes to be visible before it reads the partials.
 template <int D>
 int launch_merge(const DecodeParams& p, cudaStream_t stream) {
   const long long pairs = (long long)p.num_seqs * p.Hq;
-  decode_merge_kernel<D><<<dim3(unsigned(pairs)), dim3(kMergeWarps * 32), 0, stream>>>(p);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(pairs));
+  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, decode_merge_kernel<D>, p) != cudaSuccess) return ATTN_ERR_CUDA;
   return launch_status();
 }
 

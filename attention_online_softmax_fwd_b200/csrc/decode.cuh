@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                         const DecodeParams p) {
   static_assert(G >= 1 && G <= 16, "query heads per KV head");
   using L = DecodeSmem<D, G>;
+  launch_dependents();   // let the merge kernel be scheduled early; it waits for this grid to finish
   constexpr int NS = L::kStages;
   constexpr int KS = D / 16;   // k-steps of q.K^T
   constexpr int NT = D / 8;    // 8-column tiles of O
@@ -574,26 +575,31 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 // Combine the split partials of one (sequence, query head) per CTA: each
 // partial is a normalised O row (fp32) with its log2-sum-exp; the result is
-// sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M), M the largest lse_s. The four
-// warps take interleaved splits with several loads in flight, then combine in
-// a fixed order (deterministic).
+// sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M), M the largest lse_s. Warp w
+// takes splits w, w + 4, ... in chunks of kMergeChunk, loading each chunk's
+// lse values and O rows together (one memory round trip per chunk), and keeps a
+// running maximum; the four warps then combine in a fixed order (deterministic).
 constexpr int kMergeWarps = 4;
+constexpr int kMergeChunk = 8;   // splits per warp in flight
 template <int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const DecodeParams p) {
   constexpr int DL = D / 32;   // floats per lane: 4 (D = 128) or 2 (D = 64)
-  constexpr int kUnroll = 4;
   __shared__ float sh_m[kMergeWarps], sh_w[kMergeWarps];
   __shared__ __align__(16) float sh_acc[kMergeWarps][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seq = int(blockIdx.x / unsigned(p.Hq)), hq = int(blockIdx.x % unsigned(p.Hq));
   const int capacity = p.max_pages * p.page_size;
+  // the lengths are inputs, not results of the split kernel: read before waiting for it
   int len = __ldg(&p.seq_lens[seq]);
   len = len < 0 ? 0 : min(len, capacity);
   const int n_splits = (len + p.split_tokens - 1) / p.split_tokens;
+  // every CTA waits for the split kernel (launched as its programmatic dependent), so that this
+  // grid never completes before that one
+  grid_dependency_wait();
   __nv_bfloat16* orow = p.o + (size_t(seq) * p.Hq + hq) * D;
   const float neg_inf = -__int_as_float(0x7f800000);
   if (n_splits == 1) return;  // written by the split kernel
-  if (n_splits == 0) {
+  if (n_splits == 0) {        // a row the split kernel never writes
     for (int d = threadIdx.x; d < D; d += blockDim.x) orow[d] = __float2bfloat16_rn(0.f);
     if (p.lse && threadIdx.x == 0) p.lse[size_t(seq) * p.Hq + hq] = neg_inf;
     return;
@@ -601,65 +607,67 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const De
   const float* lse_base = p.ws_lse + size_t(seq) * p.max_splits * p.Hq + hq;
   const float* o_base = p.ws_o + (size_t(seq) * p.max_splits * p.Hq + hq) * D + lane * DL;
   const size_t o_stride = size_t(p.Hq) * D;   // floats between consecutive splits
-  // the largest partial LSE
-  float mx = neg_inf;
-  for (int s = threadIdx.x; s < n_splits; s += kMergeWarps * 32) mx = fmaxf(mx, lse_base[size_t(s) * p.Hq]);
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (lane == 0) sh_m[warp] = mx;
-  __syncthreads();
-  mx = sh_m[0];
-#pragma unroll
-  for (int w = 1; w < kMergeWarps; ++w) mx = fmaxf(mx, sh_m[w]);
-  // this warp's splits: warp, warp + 4, ...
   float acc[DL];
 #pragma unroll
   for (int d = 0; d < DL; ++d) acc[d] = 0.f;
-  float wsum = 0.f;
-  int s = warp;
-  for (; s + (kUnroll - 1) * kMergeWarps < n_splits; s += kUnroll * kMergeWarps) {
-    float ls[kUnroll], ov[kUnroll][DL];
+  float m = neg_inf, wsum = 0.f;
+  for (int base = warp; base < n_splits; base += kMergeWarps * kMergeChunk) {
+    float ls[kMergeChunk], ov[kMergeChunk][DL];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int su = s + u * kMergeWarps;
-      ls[u] = lse_base[size_t(su) * p.Hq];
-      const float* src = o_base + size_t(su) * o_stride;
-      if constexpr (DL == 4) {
-        const float4 t = *reinterpret_cast<const float4*>(src);
-        ov[u][0] = t.x; ov[u][1] = t.y; ov[u][2] = t.z; ov[u][3] = t.w;
-      } else {
-        const float2 t = *reinterpret_cast<const float2*>(src);
-        ov[u][0] = t.x; ov[u][1] = t.y;
+    for (int u = 0; u < kMergeChunk; ++u) {
+      const int su = base + u * kMergeWarps;
+      ls[u] = neg_inf;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) ov[u][d] = 0.f;
+      if (su < n_splits) {
+        ls[u] = lse_base[size_t(su) * p.Hq];
+        const float* src = o_base + size_t(su) * o_stride;
+        if constexpr (DL == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(src);
+          ov[u][0] = t.x; ov[u][1] = t.y; ov[u][2] = t.z; ov[u][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(src);
+          ov[u][0] = t.x; ov[u][1] = t.y;
+        }
       }
     }
+    float cm = ls[0];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const float w = (ls[u] == neg_inf) ? 0.f : fast_exp2(ls[u] - mx);
+    for (int u = 1; u < kMergeChunk; ++u) cm = fmaxf(cm, ls[u]);
+    if (cm > m) {   // raise the running maximum (the first finite chunk rescales zeros)
+      const float sc = (m == neg_inf) ? 0.f : fast_exp2(m - cm);
+#pragma unroll
+      for (int d = 0; d < DL; ++d) acc[d] *= sc;
+      wsum *= sc;
+      m = cm;
+    }
+#pragma unroll
+    for (int u = 0; u < kMergeChunk; ++u) {
+      const float w = (ls[u] == neg_inf) ? 0.f : fast_exp2(ls[u] - m);
       wsum += w;
 #pragma unroll
       for (int d = 0; d < DL; ++d) acc[d] = fmaf(w, ov[u][d], acc[d]);
     }
   }
-  for (; s < n_splits; s += kMergeWarps) {
-    const float ls = lse_base[size_t(s) * p.Hq];
-    const float w = (ls == neg_inf) ? 0.f : fast_exp2(ls - mx);
-    const float* src = o_base + size_t(s) * o_stride;
-    wsum += w;
-#pragma unroll
-    for (int d = 0; d < DL; ++d) acc[d] = fmaf(w, src[d], acc[d]);
-  }
 #pragma unroll
   for (int d = 0; d < DL; ++d) sh_acc[warp][lane * DL + d] = acc[d];
-  if (lane == 0) sh_w[warp] = wsum;
+  if (lane == 0) { sh_m[warp] = m; sh_w[warp] = wsum; }
   __syncthreads();
-  float wt = sh_w[0];
+  float mx = sh_m[0];
 #pragma unroll
-  for (int w = 1; w < kMergeWarps; ++w) wt += sh_w[w];
+  for (int w = 1; w < kMergeWarps; ++w) mx = fmaxf(mx, sh_m[w]);
+  float f[kMergeWarps];
+  float wt = 0.f;
+#pragma unroll
+  for (int w = 0; w < kMergeWarps; ++w) {
+    f[w] = (sh_m[w] == neg_inf) ? 0.f : fast_exp2(sh_m[w] - mx);
+    wt += f[w] * sh_w[w];
+  }
   const float inv = wt > 0.f ? 1.f / wt : 0.f;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float v = sh_acc[0][d];
+    float v = 0.f;
 #pragma unroll
-    for (int w = 1; w < kMergeWarps; ++w) v += sh_acc[w][d];
+    for (int w = 0; w < kMergeWarps; ++w) v = fmaf(f[w], sh_acc[w][d], v);
     orow[d] = __float2bfloat16_rn(v * inv);
   }
   if (p.lse && threadIdx.x == 0)

@@ -86,6 +86,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
   static_assert(G >= 1 && G <= 16, "query heads per KV head");
   static_assert(!F8 || D == 128, "the FP8 cache layout assumes 128-byte rows");
   using L = DecodeHeadsSmem<D, G, HG, F8>;
+  launch_dependents();   // let the merge kernel be scheduled early; it waits for this grid to finish
   constexpr int NS = L::kStages;
   constexpr int KS = D / 16;
   constexpr int NT = D / 8;
@@ -485,23 +486,24 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
           if (p.lse && g == 0)
             p.lse[size_t(seq) * p.Hq + hq] = lsum > 0.f ? (m_ref[c] + __log2f(lsum)) * 0.69314718055994531f : neg_inf;
         } else {
+          const uint64_t keep = l2_keep_policy();   // the merge reads these back after the KV stream
           if constexpr (F8) {
-            float4* dst = reinterpret_cast<float4*>(p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D +
-                                                    16 * g);
-            dst[0] = make_float4(o[0][c] * inv, o[1][c] * inv, o[2][c] * inv, o[3][c] * inv);
-            dst[1] = make_float4(o[4][c] * inv, o[5][c] * inv, o[6][c] * inv, o[7][c] * inv);
-            dst[2] = make_float4(o[0][c + 2] * inv, o[1][c + 2] * inv, o[2][c + 2] * inv, o[3][c + 2] * inv);
-            dst[3] = make_float4(o[4][c + 2] * inv, o[5][c + 2] * inv, o[6][c + 2] * inv, o[7][c + 2] * inv);
+            float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + 16 * g;
+            st_keep(dst, o[0][c] * inv, o[1][c] * inv, o[2][c] * inv, o[3][c] * inv, keep);
+            st_keep(dst + 4, o[4][c] * inv, o[5][c] * inv, o[6][c] * inv, o[7][c] * inv, keep);
+            st_keep(dst + 8, o[0][c + 2] * inv, o[1][c + 2] * inv, o[2][c + 2] * inv, o[3][c + 2] * inv, keep);
+            st_keep(dst + 12, o[4][c + 2] * inv, o[5][c + 2] * inv, o[6][c + 2] * inv, o[7][c + 2] * inv, keep);
           } else {
             float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + g;
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
-              dst[16 * m] = o[m][c] * inv;
-              dst[16 * m + 8] = o[m][c + 2] * inv;
+              st_keep(dst + 16 * m, o[m][c] * inv, keep);
+              st_keep(dst + 16 * m + 8, o[m][c + 2] * inv, keep);
             }
           }
           if (g == 0)
-            p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lsum > 0.f ? m_ref[c] + __log2f(lsum) : neg_inf;
+            st_keep(&p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq],
+                    lsum > 0.f ? m_ref[c] + __log2f(lsum) : neg_inf, keep);
         }
       }
     }
@@ -761,25 +763,25 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
           if (p.lse && tq == 0)
             p.lse[size_t(seq) * p.Hq + hq] = lsum > 0.f ? (m_ref[r] + __log2f(lsum)) * 0.69314718055994531f : neg_inf;
         } else {
+          const uint64_t keep = l2_keep_policy();   // the merge reads these back after the KV stream
           if constexpr (F8) {
-            float4* dst = reinterpret_cast<float4*>(p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D +
-                                                    32 * tq);
+            float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + 32 * tq;
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
               for (int n = 0; n < NT; n += 4) {
                 const int e = 2 * r + h;
-                dst[4 * h + n / 4] = make_float4(o[n][e] * inv, o[n + 1][e] * inv, o[n + 2][e] * inv,
-                                                 o[n + 3][e] * inv);
+                st_keep(dst + 16 * h + n, o[n][e] * inv, o[n + 1][e] * inv, o[n + 2][e] * inv, o[n + 3][e] * inv,
+                        keep);
               }
           } else {
             float* dst = p.ws_o + ((size_t(seq) * p.max_splits + split) * p.Hq + hq) * D + 2 * tq;
 #pragma unroll
-            for (int n = 0; n < NT; ++n)
-              *reinterpret_cast<float2*>(dst + n * 8) = make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+            for (int n = 0; n < NT; ++n) st_keep(dst + n * 8, o[n][2 * r] * inv, o[n][2 * r + 1] * inv, keep);
           }
           if (tq == 0)
-            p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq] = lsum > 0.f ? m_ref[r] + __log2f(lsum) : neg_inf;
+            st_keep(&p.ws_lse[(size_t(seq) * p.max_splits + split) * p.Hq + hq],
+                    lsum > 0.f ? m_ref[r] + __log2f(lsum) : neg_inf, keep);
         }
       }
     }

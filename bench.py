@@ -351,7 +351,7 @@ def run_gpu(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel<128,causal>", "achieved": pre_tfs,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": pre_tfs / peaks["bf16_tflops"],
                      "peak_source": f"{peak_src} bf16 burst", "traffic": traffic.get("prefill_bytes_per_launch")},
-        "roofline_decode": {"bound": "hbm", "kernel": "decode_heads_kernel<128,4,8>+decode_merge_kernel",
+        "roofline_decode": {"bound": "hbm", "kernel": "decode_heads_kernel<128,4,4>+decode_merge_kernel",
                             "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": dec_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy",
                             "traffic": traffic.get("decode_bytes_per_call")},
@@ -364,10 +364,11 @@ def run_gpu(args, world, rank, local):
         "wall_s_timed_region": wall,
         "outputs_finite": finite,
     }
+    if rank == 0 and world == 1 and not args.no_extras:
+        line["decode_fp8"] = fp8_decode_report(dev, peaks, cache, flush)
+        line["chunked_prefill_paged"] = chunked_prefill_report(dev, peaks)
     if rank == 0 and world == 1 and not args.no_blasst:
         line["blasst_long_context"] = blasst_long_context_report(dev)
-        line["chunked_prefill_paged"] = chunked_prefill_report(dev, peaks)
-        line["decode_fp8"] = fp8_decode_report(dev, peaks, cache, flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfs, gbs, secs, desc = oracle_sample(int(args.cpu_heads), 4)
         line["cpu_baseline"] = {"value": tfs, "unit": "TFLOP/s", "cores": cpu_threads()[0], "kind": "oracle",
@@ -412,7 +413,7 @@ def fp8_decode_report(dev, peaks, cache, flush, reps=10):
     by = decode_bytes(cache.seq_lens.tolist(), dc["Hq"], dc["Hkv"], dc["D"], cache.max_pages, kv_elem_bytes=1)
     gbs = by / (ms * 1e-3) / 1e9
     return {"workload": f"{DECODE_CFG} with E4M3 K/V pools, split {DECODE_SPLIT}",
-            "kernel": "decode_heads_kernel<128,4,8,fp8>+decode_merge_kernel", "ms": ms, "gbs": gbs,
+            "kernel": "decode_heads_kernel<128,4,4,fp8>+decode_merge_kernel", "ms": ms, "gbs": gbs,
             "bytes_per_call": by, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
             "frac_of_spec_8000": gbs / SPEC_PEAKS["hbm_gbs"],
             "tokens_per_s": int(cache.seq_lens.sum()) / (ms * 1e-3)}
@@ -539,6 +540,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-blasst", action="store_true", help="skip the long-context BLASST report")
+    ap.add_argument("--no-extras", action="store_true", help="skip the FP8-decode and chunked-prefill reports")
     ap.add_argument("--cpu-heads", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3:
