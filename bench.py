@@ -415,6 +415,7 @@ def fp8_decode_report(dev, peaks, cache, flush, reps=10):
     return {"workload": f"{DECODE_CFG} with E4M3 K/V pools, split {DECODE_SPLIT}",
             "kernel": "decode_heads_kernel<128,4,4,fp8>+decode_merge_kernel", "ms": ms, "gbs": gbs,
             "bytes_per_call": by, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
+            "traffic": load_profile_traffic().get("decode_fp8_bytes_per_call"),
             "frac_of_spec_8000": gbs / SPEC_PEAKS["hbm_gbs"],
             "tokens_per_s": int(cache.seq_lens.sum()) / (ms * 1e-3)}
 
