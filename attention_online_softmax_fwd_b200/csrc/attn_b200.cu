@@ -432,9 +432,10 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
   const int hg = G <= 8 ? (Hkv % 4 == 0 ? 4 : 0) : (Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0));
   if (!use_skip && hg > 0) {
     // dense: one item per group of hg KV heads, 16-token stages covering all of them
-    const uint64_t hdims[5] = {64, uint64_t(D / 64), uint64_t(page_size), uint64_t(Hkv), uint64_t(num_pages)};
-    const uint64_t hstrides[4] = {128, uint64_t(Hkv) * D * 2, uint64_t(D) * 2, uint64_t(page_size) * Hkv * D * 2};
-    const uint32_t hbox[5] = {64, uint32_t(D / 64), uint32_t(kDhChunk), uint32_t(hg), 1};
+    // {64 columns, token, 64-column half, head, page}: a head's 16 tokens land as [half][token][64]
+    const uint64_t hdims[5] = {64, uint64_t(page_size), uint64_t(D / 64), uint64_t(Hkv), uint64_t(num_pages)};
+    const uint64_t hstrides[4] = {uint64_t(Hkv) * D * 2, 128, uint64_t(D) * 2, uint64_t(page_size) * Hkv * D * 2};
+    const uint32_t hbox[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), uint32_t(hg), 1};
     CUtensorMap hk, hv;
     if (int st = encode_map5(&hk, k_pages, hdims, hstrides, hbox)) return st;
     if (int st = encode_map5(&hv, v_pages, hdims, hstrides, hbox)) return st;

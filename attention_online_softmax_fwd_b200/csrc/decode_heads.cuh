@@ -69,6 +69,16 @@ struct DecodeHeadsSmem {
   static_assert(kStages >= 2, "ring depth");
 };
 
+// Byte offset of 16-byte chunk `c` (0 .. D/8 - 1) of token `t` (0 .. 15) in one head's
+// bf16 block of a stage. The copy orders the block [64-column half][token][64 columns]:
+// 128-byte row (c / 8) * 16 + t, unit (c mod 8) XOR t mod 8, so eight consecutive
+// tokens of one half sit in eight different bank groups.
+template <int D>
+__device__ __forceinline__ uint32_t dh_swz(int t, int c) {
+  const int row = (c >> 3) * kDhChunk + t;
+  return uint32_t(row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
+
 // item -> (split, seq, group): splits outermost so that full-length splits go first
 __device__ __forceinline__ void dh_item_coords(long long item, int num_seqs, int n_groups, int& seq, int& split,
                                                int& grp) {
@@ -212,8 +222,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
               tma_load_4d(kdst, &tm_k, &full[slot], 0, in_page, grp * HG, page[h]);
               tma_load_4d(kdst + L::kKVBytes, &tm_v, &full[slot], 0, in_page, grp * HG, page[h]);
             } else {
-              tma_load_5d(kdst, &tm_k, &full[slot], 0, 0, in_page, grp * HG, page[h]);
-              tma_load_5d(kdst + L::kKVBytes, &tm_v, &full[slot], 0, 0, in_page, grp * HG, page[h]);
+              tma_load_5d(kdst, &tm_k, &full[slot], 0, in_page, 0, grp * HG, page[h]);
+              tma_load_5d(kdst + L::kKVBytes, &tm_v, &full[slot], 0, in_page, 0, grp * HG, page[h]);
             }
           }
         }
@@ -322,7 +332,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
             uint32_t af[KS][4];
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks)
-              ldsm_x4(kaddr + swz_off<D>(tok, ks * 2 + (mi >> 1)), af[ks][0], af[ks][1], af[ks][2], af[ks][3]);
+              ldsm_x4(kaddr + dh_swz<D>(tok, ks * 2 + (mi >> 1)), af[ks][0], af[ks][1], af[ks][2], af[ks][3]);
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) mma_bf16_16816(sp[ks & 1], af[ks], qb[ks][0], qb[ks][1]);
           }
@@ -405,7 +415,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
             uint32_t a[4];
-            ldsm_x4_t(vaddr + swz_off<D>(tok, 2 * m + (mi & 1)), a[0], a[1], a[2], a[3]);
+            ldsm_x4_t(vaddr + dh_swz<D>(tok, 2 * m + (mi & 1)), a[0], a[1], a[2], a[3]);
             a[0] &= mk0; a[1] &= mk0; a[2] &= mk1; a[3] &= mk1;
             mma_bf16_16816(o[m], a, pb[0][0], pb[0][1]);
           }
@@ -593,7 +603,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
             uint32_t bfr[KS][4];
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks)
-              ldsm_x4(kaddr + swz_off<D>(tok, ks * 2 + (mi & 1)), bfr[ks][0], bfr[ks][1], bfr[ks][2], bfr[ks][3]);
+              ldsm_x4(kaddr + dh_swz<D>(tok, ks * 2 + (mi & 1)), bfr[ks][0], bfr[ks][1], bfr[ks][2], bfr[ks][3]);
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
               mma_bf16_16816(sp[0][ks & 1], qa[ks], bfr[ks][0], bfr[ks][1]);
@@ -626,7 +636,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
           // zero the V rows of tokens past the end so that 0 * (stale or NaN) cannot reach O
           for (int t = ntok; t < kDhChunk; ++t)
             for (int c = lane; c < D / 8; c += 32)
-              *reinterpret_cast<uint4*>(stage + L::kKVBytes + warp * L::kHeadBytes + swz_off<D>(t, c)) =
+              *reinterpret_cast<uint4*>(stage + L::kKVBytes + warp * L::kHeadBytes + dh_swz<D>(t, c)) =
                   make_uint4(0, 0, 0, 0);
           __syncwarp();
         }
@@ -713,7 +723,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
 #pragma unroll
           for (int n2 = 0; n2 < NT / 2; ++n2) {
             uint32_t v0, v1, v2, v3;
-            ldsm_x4_t(vaddr + swz_off<D>(tok, n2 * 2 + (mi >> 1)), v0, v1, v2, v3);
+            ldsm_x4_t(vaddr + dh_swz<D>(tok, n2 * 2 + (mi >> 1)), v0, v1, v2, v3);
             mma_bf16_16816(o[2 * n2], pa, v0, v1);
             mma_bf16_16816(o[2 * n2 + 1], pa, v2, v3);
           }
