@@ -4,6 +4,7 @@
 // attn_read_device_status, which is documented to).
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -96,6 +97,28 @@ int encode_map5(CUtensorMap* map, const void* base, const uint64_t dims[5], cons
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Once per device and kernel (one mask per kernel, keyed by the kernel itself): check that it
+// was compiled with at least `min_regs` registers per thread (0: no check) and raise its
+// dynamic shared-memory limit. The launch path then makes no attribute call, which keeps it
+// a plain sequence of stream operations under graph capture and saves host time per launch.
+template <auto kernel>
+int set_smem_once(int smem, int min_regs = 0) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return ATTN_OK;
+  if (min_regs > 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (attr.numRegs < min_regs) return ATTN_ERR_UNSUPPORTED;
+  }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return ATTN_OK;
+}
+
 // [B][S][H][D] bf16 tensor as a 4-D map {D, S, H, B}; box = 64 columns x 128 rows of one head.
 int encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
   const uint64_t dims[4] = {uint64_t(D), uint64_t(S), uint64_t(H), uint64_t(B)};
@@ -112,12 +135,11 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   auto kernel = prefill_kernel<D, CAUSAL, SKIP, PAGED>;
   constexpr int smem = PrefillSmem<D>::kDynamic;
   // The kernel moves registers between warpgroups with setmaxnreg; the block's
-  // launch allocation must cover the split or the increase would never return.
-  cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (attr.numRegs * kPfThreads < kPfRegPoolNeeded) return ATTN_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  // launch allocation must cover the split or the increase would never return
+  // (checked with the shared-memory limit, once per device).
+  if (int st = set_smem_once<prefill_kernel<D, CAUSAL, SKIP, PAGED>>(smem, (kPfRegPoolNeeded + kPfThreads - 1) /
+                                                                            kPfThreads))
+    return st;
   const long long grid = p.num_items < sms ? p.num_items : sms;
   kernel<<<dim3(unsigned(grid)), dim3(kPfThreads), smem, stream>>>(tq, tk, tv, p);
   return launch_status();
@@ -220,8 +242,7 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodePara
                   cudaStream_t stream) {
   auto kernel = decode_split_kernel<D, G, SKIP>;
   constexpr int smem = DecodeSmem<D, G>::kDynamic;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (int st = set_smem_once<decode_split_kernel<D, G, SKIP>>(smem)) return st;
   const long long grid = p.num_items < sms ? p.num_items : sms;
   kernel<<<dim3(unsigned(grid)), dim3(kDecThreads), smem, stream>>>(tk, tv, p);
   if (int st = launch_status()) return st;
@@ -246,8 +267,7 @@ int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
                         int sms, cudaStream_t stream) {
   auto kernel = decode_heads_kernel<D, G, HG, F8>;
   constexpr int smem = DecodeHeadsSmem<D, G, HG, F8>::kDynamic;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (int st = set_smem_once<decode_heads_kernel<D, G, HG, F8>>(smem)) return st;
   const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
   const long long slots = (long long)sms * DecodeHeadsSmem<D, G, HG, F8>::kBlocks;
   const long long grid = items < slots ? items : slots;
