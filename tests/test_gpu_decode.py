@@ -29,7 +29,7 @@ def _run(cache, dev, split, lam=None):
 
 
 @pytest.mark.parametrize("Hq,Hkv,D", [(8, 2, 128), (8, 8, 64), (16, 1, 128), (4, 2, 64), (32, 16, 128),
-                                      (16, 2, 128)])
+                                      (16, 2, 128), (24, 12, 128), (48, 12, 64), (128, 8, 128), (64, 4, 64)])
 @pytest.mark.parametrize("page_size", [16, 64, 256])
 def test_decode_small(cuda_device, Hq, Hkv, D, page_size):
     lens = [1, 63, 64, 65, 700, 2049, 0, 130]

@@ -27,7 +27,7 @@ def _run(cache, kc, ks, vc, vs, dev, split, status=None):
     return o, lse, scale
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(8, 4), (32, 8), (16, 16), (64, 8), (128, 8), (4, 4)])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 4), (32, 8), (16, 16), (64, 8), (128, 8), (4, 4), (24, 12), (64, 4)])
 @pytest.mark.parametrize("page_size", [16, 64, 256])
 def test_decode_fp8_small(cuda_device, Hq, Hkv, page_size):
     lens = [1, 15, 16, 17, 63, 700, 2049, 0, 130]
