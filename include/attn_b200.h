@@ -21,15 +21,20 @@
  * PART03). Hkv == Hq is MHA, Hkv == 1 is MQA.
  *
  * Optional BLASST tile skip ("高效部署稀疏注意力加速方案：BLASST方法详解与实践指南",
- * 架构与组件): with lambda > 0, a tile of 64 keys is skipped -- no exponentials,
- * no V load, no P V product -- when exp(tile_rowmax - running_max) < lambda for
- * every row of its decision unit. The running maximum is over the unit's tiles
- * already kept, in ascending key order. lambda == 0 computes the dense result.
+ * 架构与组件): with lambda > 0, a tile of 64 keys is skipped -- no P V product, and
+ * no exponentials wherever the decision is known before they would be computed --
+ * when exp(tile_rowmax - running_max) < lambda for every row of its decision unit.
+ * (The V tile is still read in this version: it travels with K.) The running
+ * maximum is over the unit's tiles already kept, in ascending key order.
+ * lambda == 0 computes the dense result.
  *
  * Common conventions
  *   - Every pointer is a DEVICE pointer owned by the caller. The library never
  *     allocates, frees or synchronises; all work is enqueued on `stream`
- *     (a cudaStream_t; NULL is the legacy default stream).
+ *     (a cudaStream_t; NULL is the legacy default stream). A call enqueues only
+ *     kernel launches (and, for decode, one small memset); kernel attributes are
+ *     set at a function's first call on a device. After one eager call, the
+ *     calls can be captured into a CUDA graph and replayed.
  *   - bf16 means IEEE bfloat16 (__nv_bfloat16), row-major, contiguous.
  *     Accumulation is fp32. LSE is the natural-log log-sum-exp of the scaled
  *     scores, fp32.
