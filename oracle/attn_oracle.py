@@ -42,6 +42,9 @@ What it computes, and the passages it follows:
 * Writing new tokens' K/V into the paged cache (kv_append).
 * FP8 E4M3 paged cache with one scale per pool (decode_paged_fp8): the
   reading stated in its docstring; E4M3 decoded from its bit layout.
+* The exact formula restricted to the tiles that a given decision mask keeps
+  (prefill_with_skip_mask, decode_paged_with_skip_mask), for decision sets
+  that differ from the walk's only where a decision sits within the tie band.
 
 Parity status: dense prefill, paged decode, chunked paged prefill and the
 gather are pinned by the
@@ -425,3 +428,69 @@ def decode_paged_blasst(q, k_pages, v_pages, block_table, seq_lens, page_size: i
                 o[b, rows, :] = ob
                 lse[b, rows] = lb
     return o, lse, skip, margin
+
+
+def prefill_with_skip_mask(q, k, v, causal: bool, scale: float, skip_mask, heads=None, q_tiles=None):
+    """Prefill restricted to the tiles a given decision mask keeps.
+
+    The same decision units and tiles as prefill_blasst, but the decisions are
+    read from ``skip_mask`` [B, Hq, ceil(S/128), ceil(S/64)] (1 skipped, 0 kept,
+    2 not visited) instead of being walked: every visible key of a tile whose
+    entry is not 1 takes part in the exact formula. This evaluates a decision
+    set that differs from the walk's own inside the tie band of a decision.
+    Returns o [B,S,Hq,D], lse [B,Hq,S] (NaN outside the sample).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    mask = np.asarray(skip_mask.cpu() if hasattr(skip_mask, "cpu") else skip_mask)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    n_qt = -(-S // Q_TILE)
+    o = np.full((B, S, Hq, v.shape[-1]), np.nan)
+    lse = np.full((B, Hq, S), np.nan)
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(Hq)]
+    for b, hq in heads:
+        kv = kv_head_of(hq, Hq, Hkv)
+        for qt in (range(n_qt) if q_tiles is None else q_tiles):
+            rows = np.arange(qt * Q_TILE, min(qt * Q_TILE + Q_TILE, S))
+            vis = causal_visible(rows, S) if causal else np.ones((len(rows), S), bool)
+            key_tile = np.arange(S) // KV_TILE
+            kept = vis & (mask[b, hq, qt, key_tile] != 1)[None, :]
+            ob, lb = attention_rows(q[b, rows, hq, :], k[b, :, kv, :], v[b, :, kv, :], scale, kept)
+            o[b, rows, hq, :] = ob
+            lse[b, hq, rows] = lb
+    return o, lse
+
+
+def decode_paged_with_skip_mask(q, k_pages, v_pages, block_table, seq_lens, page_size: int, scale: float,
+                                skip_mask, rows_per_unit: str = "group", seqs=None):
+    """Paged decode restricted to the tiles a given decision mask keeps.
+
+    ``skip_mask`` [N, Hkv, max_tiles] (rows_per_unit="group") or [N, Hq,
+    max_tiles] ("head"), 1 skipped / 0 kept / 2 not visited, as returned by
+    decode_paged_blasst: each query head attends to the tokens of the 64-token
+    tiles its unit keeps. Returns o [N,Hq,D], lse [N,Hq].
+    """
+    q = _f64(q)
+    mask = np.asarray(skip_mask.cpu() if hasattr(skip_mask, "cpu") else skip_mask)
+    bt = np.asarray(block_table)
+    lens = np.asarray(seq_lens)
+    N, Hq, D = q.shape
+    Hkv = k_pages.shape[2]
+    o = np.full((N, Hq, D), np.nan)
+    lse = np.full((N, Hq), np.nan)
+    for b in (range(N) if seqs is None else seqs):
+        L = int(lens[b])
+        if L == 0:
+            o[b], lse[b] = 0.0, NEG_INF
+            continue
+        kb = gather_pages(k_pages, bt[b], L, page_size)
+        vb = gather_pages(v_pages, bt[b], L, page_size)
+        tile = np.arange(L) // KV_TILE
+        for hq in range(Hq):
+            kv = kv_head_of(hq, Hq, Hkv)
+            unit = kv if rows_per_unit == "group" else hq
+            kept = (mask[b, unit, tile] != 1)[None, :]
+            ob, lb = attention_rows(q[b, hq][None, :], kb[:, kv, :], vb[:, kv, :], scale, kept)
+            o[b, hq], lse[b, hq] = ob[0], lb[0]
+    return o, lse

@@ -10,12 +10,34 @@ import torch
 import attention_online_softmax_fwd_b200 as ab
 from attention_online_softmax_fwd_b200 import inputs as gen
 from oracle import attn_oracle as orc
-from parity_util import compare_output, compare_skip
+from parity_util import compare_blasst, compare_output
 
 pytestmark = pytest.mark.gpu
 
 C = gen.CONFIGS["blasst_long_context"]
 SPLIT = 2048
+
+
+def _check_units(q, k, v, scale, o, lse, mask, o_ref, lse_ref, m_ref, margin, heads, q_tiles, label):
+    """Decisions and outputs of sampled prefill units (b, hq, 128-row query tile);
+    a decision that went the other way inside the tie band is checked on the
+    GPU's own decisions. Returns the skipped counts (oracle, GPU)."""
+    mg = mask.cpu().numpy()
+    og, lg = o.cpu(), lse.cpu()
+    skipped = skipped_gpu = 0
+    for b, h in heads:
+        for qt in q_tiles:
+            rows = list(range(qt * 128, min(qt * 128 + 128, q.shape[1])))
+
+            def with_gpu_mask(_unit_mask, b=b, h=h, qt=qt, rows=rows):
+                of, lf = orc.prefill_with_skip_mask(q, k, v, True, scale, mg, heads=[(b, h)], q_tiles=[qt])
+                return of[b, rows, h], lf[b, h, rows]
+
+            st = compare_blasst(og[b, rows, h], lg[b, h, rows], mg[b, h, qt], o_ref[b, rows, h], lse_ref[b, h, rows],
+                                m_ref[b, h, qt], margin[b, h, qt], with_gpu_mask, label=f"{label} h={h} qt={qt}")
+            skipped += st["skipped"]
+            skipped_gpu += st["skipped_gpu"]
+    return skipped, skipped_gpu
 
 
 @pytest.fixture(scope="module")
@@ -35,15 +57,9 @@ def test_long_context_prefill(cuda_device, workload, lam):
     heads = [(0, 3), (0, 30)]
     q_tiles = [0, 77, 255]
     o_ref, lse_ref, m_ref, margin = orc.prefill_blasst(q, k, v, True, scale, lam, heads=heads, q_tiles=q_tiles)
-    mg = mask.cpu().numpy()
-    og, lg = o.cpu(), lse.cpu()
-    for b, h in heads:
-        for qt in q_tiles:
-            st = compare_skip(mg[b, h, qt], m_ref[b, h, qt], margin[b, h, qt], label=f"h={h} qt={qt}")
-            rows = list(range(qt * 128, qt * 128 + 128))
-            if st["tie_mismatches"] == 0:
-                compare_output(og[b, rows, h], o_ref[b, rows, h], lg[b, h, rows], lse_ref[b, h, rows],
-                               label=f"lam={lam} h={h} qt={qt}")
+    skipped, skipped_gpu = _check_units(q, k, v, scale, o, lse, mask, o_ref, lse_ref, m_ref, margin, heads, q_tiles,
+                                        f"lam={lam}")
+    print(f"prefill lam={lam}: sampled units skipped {skipped} (GPU {skipped_gpu})")
     if lam == 0.0:
         assert not (mask == 1).any()
 
@@ -59,10 +75,22 @@ def test_long_context_decode(cuda_device, workload, lam):
     o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages,
                                                             cache.block_table, cache.seq_lens, C["page_size"],
                                                             scale, lam, SPLIT)
-    st = compare_skip(mask, m_ref, margin, label=f"decode lam={lam}")
-    if st["tie_mismatches"] == 0:
-        compare_output(o, o_ref, lse, lse_ref, label=f"decode lam={lam}")
-    print(f"decode lam={lam}: skipped {st['skipped']} of {st['decisions']} tiles")
+    st = compare_blasst(o, lse, mask, o_ref, lse_ref, m_ref, margin, _decode_with_mask(cache, scale),
+                        label=f"decode lam={lam}")
+    print(f"decode lam={lam}: skipped {st['skipped']} of {st['decisions']} tiles (GPU {st['skipped_gpu']}, "
+          f"{st['ties']} within the tie band)")
+    # the skipped fraction is the oracle's up to decisions inside the tie band
+    assert abs(st["skipped_gpu"] - st["skipped"]) <= st["tie_mismatches"]
+    if lam == 0.3:
+        assert st["skipped"] > 0
+
+
+def _decode_with_mask(cache, scale, rows_per_unit="group"):
+    def f(mask):
+        return orc.decode_paged_with_skip_mask(cache.q, cache.k_pages, cache.v_pages, cache.block_table,
+                                               cache.seq_lens, C["page_size"], scale, mask,
+                                               rows_per_unit=rows_per_unit)
+    return f
 
 
 def test_long_context_decode_equals_prefill_last_row(cuda_device, workload):
@@ -84,10 +112,6 @@ def test_long_context_decode_equals_prefill_last_row(cuda_device, workload):
 def dominant():
     q, k, v = gen.peaked_prefill_inputs(C["B"], C["Hq"], C["Hkv"], C["S"], C["D"], C["seed"] + 7, amp=12.0,
                                         period=C["S"])
-    # with ~99% of tiles dropped the output is close to V's row 0; V is scaled
-    # down so that the bf16 rounding of the output alone stays well inside the
-    # mean tolerance
-    v = (v.float() * 0.25).to(torch.bfloat16)
     cache = gen.paged_from_contiguous(q[:, C["S"] - 1], k, v, page_size=C["page_size"], seed=C["seed"] + 8)
     return q, k, v, cache
 
@@ -102,17 +126,8 @@ def test_long_context_dominant_key_prefill(cuda_device, dominant, lam):
     heads = [(0, 5), (0, 17)]
     q_tiles = [1, 130, 255]
     o_ref, lse_ref, m_ref, margin = orc.prefill_blasst(q, k, v, True, scale, lam, heads=heads, q_tiles=q_tiles)
-    mg = mask.cpu().numpy()
-    og, lg = o.cpu(), lse.cpu()
-    skipped = 0
-    for b, h in heads:
-        for qt in q_tiles:
-            st = compare_skip(mg[b, h, qt], m_ref[b, h, qt], margin[b, h, qt], label=f"h={h} qt={qt}")
-            skipped += st["skipped"]
-            rows = list(range(qt * 128, qt * 128 + 128))
-            if st["tie_mismatches"] == 0:
-                compare_output(og[b, rows, h], o_ref[b, rows, h], lg[b, h, rows], lse_ref[b, h, rows],
-                               label=f"dominant lam={lam} h={h} qt={qt}")
+    skipped, _ = _check_units(q, k, v, scale, o, lse, mask, o_ref, lse_ref, m_ref, margin, heads, q_tiles,
+                              f"dominant lam={lam}")
     assert skipped > 0.9 * sum(min(2 * qt + 2, C["S"] // 64) for qt in q_tiles) * len(heads)
 
 
@@ -127,7 +142,6 @@ def test_long_context_dominant_key_decode(cuda_device, dominant, split):
     o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(cache.q, cache.k_pages, cache.v_pages,
                                                             cache.block_table, cache.seq_lens, C["page_size"],
                                                             scale, 0.1, split)
-    st = compare_skip(mask, m_ref, margin, label=f"dominant decode split={split}")
+    st = compare_blasst(o, lse, mask, o_ref, lse_ref, m_ref, margin, _decode_with_mask(cache, scale),
+                        label=f"dominant decode split={split}")
     assert st["skipped"] > 0
-    if st["tie_mismatches"] == 0:
-        compare_output(o, o_ref, lse, lse_ref, label=f"dominant decode split={split}")

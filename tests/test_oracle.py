@@ -593,3 +593,86 @@ def test_fp8_decode_is_decode_of_the_dequantised_cache():
     np.testing.assert_array_equal(lse, ld)
     assert np.isfinite(o).all()                   # poisoned (NaN) slots are never read
 
+
+
+# ---------------------------------------------------------------- the formula on a given decision mask
+
+def brute_prefill_masked(q, k, v, causal, scale, skip_mask):
+    """Scalar loops: row i of head h sees key j iff j is visible and the 64-key
+    tile of j is not marked skipped (1) for the 128-row tile of i."""
+    B, S, Hq, D = q.shape
+    G = Hq // k.shape[2]
+    o = np.zeros((B, S, Hq, D))
+    lse = np.zeros((B, Hq, S))
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(S):
+                w = []
+                for j in range(S):
+                    if (causal and j > i) or skip_mask[b, h, i // 128, j // 64] == 1:
+                        continue
+                    s = sum(q[b, i, h, d] * k[b, j, h // G, d] for d in range(D)) * scale
+                    w.append((j, math.exp(s)))
+                z = sum(e for _, e in w)
+                for d in range(D):
+                    o[b, i, h, d] = sum(e * v[b, j, h // G, d] for j, e in w) / z
+                lse[b, h, i] = math.log(z)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_with_skip_mask_matches_brute_force(causal):
+    B, Hq, Hkv, S, D = 1, 2, 1, 150, 3
+    q, k, v = _rand((B, S, Hq, D), 71), _rand((B, S, Hkv, D), 72), _rand((B, S, Hkv, D), 73)
+    rng = np.random.default_rng(74)
+    mask = rng.integers(0, 2, (B, Hq, 2, 3)).astype(np.uint8)
+    mask[..., 0] = 0            # every row keeps a key of its first tile
+    o, lse = orc.prefill_with_skip_mask(q, k, v, causal, 0.5, mask)
+    ob, lb = brute_prefill_masked(q, k, v, causal, 0.5, mask)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lb, rtol=0, atol=1e-12)
+
+
+def test_prefill_with_skip_mask_keep_all_is_dense_and_walk_mask_is_walk():
+    q, k, v = _peaked(1, 4, 2, 300, 16, 171, amp=8.0, period=1 << 20)
+    for causal in (True, False):
+        keep = np.zeros((1, 4, 3, 5), np.uint8)
+        o, lse = orc.prefill_with_skip_mask(q, k, v, causal, 0.25, keep)
+        od, ld = orc.prefill(q, k, v, causal, 0.25)
+        np.testing.assert_allclose(o, od, atol=1e-12)
+        np.testing.assert_allclose(lse, ld, atol=1e-12)
+        ow, lw, skip, _ = orc.prefill_blasst(q, k, v, causal, 0.25, 0.3)
+        assert skip.shape == keep.shape and (skip == 1).any()
+        om, lm = orc.prefill_with_skip_mask(q, k, v, causal, 0.25, skip)
+        np.testing.assert_allclose(om, ow, atol=1e-12)
+        np.testing.assert_allclose(lm, lw, atol=1e-12)
+
+
+def test_decode_with_skip_mask_matches_brute_force():
+    S, Hq, Hkv, D = 300, 4, 2, 8
+    q, k, v = gen.peaked_prefill_inputs(1, Hq, Hkv, S, D, seed=181, amp=6.0)
+    cache = gen.paged_from_contiguous(q[:, S - 1], k, v, page_size=16, seed=182)
+    rng = np.random.default_rng(183)
+    n_tiles = -(-cache.max_pages * 16 // 64)
+    scale = 0.3
+    qd, kd, vd = cache.q.double().numpy(), k[0].double().numpy(), v[0].double().numpy()
+    for unit_rows, n_units in (("group", Hkv), ("head", Hq)):
+        mask = rng.integers(0, 2, (1, n_units, n_tiles)).astype(np.uint8)
+        mask[..., 0] = 0
+        o, lse = orc.decode_paged_with_skip_mask(cache.q, cache.k_pages, cache.v_pages, cache.block_table,
+                                                 cache.seq_lens, 16, scale, mask, rows_per_unit=unit_rows)
+        for h in range(Hq):
+            kv = h // (Hq // Hkv)
+            unit = kv if unit_rows == "group" else h
+            w = [(j, math.exp(scale * sum(qd[0, h, d] * kd[j, kv, d] for d in range(D))))
+                 for j in range(S) if mask[0, unit, j // 64] != 1]
+            z = sum(e for _, e in w)
+            for d in range(D):
+                assert abs(o[0, h, d] - sum(e * vd[j, kv, d] for j, e in w) / z) < 1e-12
+            assert abs(lse[0, h] - math.log(z)) < 1e-12
+    keep = np.zeros((1, Hkv, n_tiles), np.uint8)
+    o, lse = orc.decode_paged_with_skip_mask(cache.q, cache.k_pages, cache.v_pages, cache.block_table,
+                                             cache.seq_lens, 16, scale, keep)
+    od, ld = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens, 16, scale)
+    np.testing.assert_allclose(o, od, atol=1e-12)
+    np.testing.assert_allclose(lse, ld, atol=1e-12)

@@ -17,7 +17,6 @@ import torch
 
 from attention_online_softmax_fwd_b200 import binding
 from attention_online_softmax_fwd_b200 import inputs as gen
-from parity_util import compare_output
 
 pytestmark = pytest.mark.gpu
 
@@ -59,8 +58,8 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_device):
         assert _noalloc_call(lib, cache, cuda_device, split, o, lse) == 0
         o_ref, lse_ref = _workspace_call(cache, cuda_device, split)
         torch.cuda.synchronize()
-        compare_output(o, o_ref.float().cpu().double().numpy(), lse, lse_ref.cpu().double().numpy(),
-                       label=f"noalloc split={split}")
+        # the same kernels on the same inputs, in a fixed order: the results agree bit for bit
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref), f"noalloc split={split}"
         assert torch.isfinite(o.float()).all()
 
 
