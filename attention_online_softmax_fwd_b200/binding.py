@@ -44,19 +44,23 @@ SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_abi_version": (_I, []),
     "attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
-    "attn_prefill_blasst": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P]),
+    "attn_prefill_blasst": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P]),
     "attn_prefill_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
     "attn_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "attn_decode_blasst_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
-                               _P, _SZ, _P, _P, _P]),
+                               _P, _SZ, _P, _P, _P, _P]),
     "attn_decode_paged_blasst_heads": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P,
-                                            _P, _P, _SZ, _P, _P, _P]),
+                                            _P, _P, _SZ, _P, _P, _P, _P]),
     "attn_kv_append": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "attn_decode_paged_fp8": (_I, [_P, _P, _P, _F, _F, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P,
                                    _P, _SZ, _P, _P]),
     "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                        _P, _P, _P]),
     "attn_read_device_status": (_I, [ctypes.POINTER(_I), _I]),
+    "attn_set_library_status": (_I, [_I]),
+    "attn_debug_prefill_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, ctypes.c_ulonglong, _I,
+                                        _P, _P]),
 }
 
 NOALLOC_SCRATCH_BYTES = 16 << 20   # ATTN_NOALLOC_SCRATCH_BYTES
@@ -108,10 +112,26 @@ def default_scale(D: int) -> float:
 
 
 def read_device_status(clear: bool = True) -> int:
-    """Library-wide device status word (synchronises the device)."""
+    """Library-wide device status word (synchronises the device); written only
+    while set_library_status(True) is in effect on the device."""
     out = ctypes.c_int(0)
     _check(load_library().attn_read_device_status(ctypes.byref(out), int(clear)), "attn_read_device_status")
     return out.value
+
+
+def set_library_status(enable: bool) -> None:
+    """Switch the library's device status word on the current device on or off."""
+    _check(load_library().attn_set_library_status(int(bool(enable))), "attn_set_library_status")
+
+
+def _counter(t, name):
+    """A one-element int64 device tensor used as the library's unsigned 64-bit counter."""
+    if t is None:
+        return None
+    _need(t, torch.int64, 1, name)
+    if t.numel() != 1:
+        raise AttnError(f"{name}: expected one element")
+    return t
 
 
 # ------------------------------------------------------------------ prefill
@@ -188,10 +208,13 @@ def prefill_skip_mask_shape(B, Hq, S):
 
 
 def prefill_blasst(q, k, v, lam: float, causal: bool = True, scale: float | None = None, out=None,
-                   lse=None, skip_mask=True, device_status=None, return_lse: bool = True, stream=None):
+                   lse=None, skip_mask=True, device_status=None, return_lse: bool = True, stream=None,
+                   skipped_tiles=None):
     """Prefill with the BLASST tile skip. Returns (o, lse, skip_mask) where
     skip_mask [B, Hq, ceil(S/128), ceil(S/64)] uint8 holds 1 (skipped) / 0 (kept)
-    for visited tiles and 2 for tiles never visited."""
+    for visited tiles and 2 for tiles never visited. ``skipped_tiles`` (a
+    one-element int64 device tensor) receives the count of skipped decisions
+    added to its value."""
     B, S, Hq, Hkv, D, o, lse = _prefill_args(q, k, v, out, lse, return_lse)
     scale = default_scale(D) if scale is None else scale
     mask = None
@@ -200,7 +223,8 @@ def prefill_blasst(q, k, v, lam: float, causal: bool = True, scale: float | None
     elif isinstance(skip_mask, torch.Tensor):
         mask = skip_mask
     st = load_library().attn_prefill_blasst(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, S, D,
-                                            int(bool(causal)), scale, lam, _ptr(mask), _ptr(device_status),
+                                            int(bool(causal)), scale, lam, _ptr(mask),
+                                            _ptr(_counter(skipped_tiles, "skipped_tiles")), _ptr(device_status),
                                             _stream_handle(stream))
     _check(st, "attn_prefill_blasst")
     return o, lse, mask
@@ -209,7 +233,14 @@ def prefill_blasst(q, k, v, lam: float, causal: bool = True, scale: float | None
 # ------------------------------------------------------------------ decode
 
 def decode_workspace_bytes(num_seqs, Hq, D, max_pages, page_size, split_tokens) -> int:
+    """Workspace of the dense decode."""
     return int(load_library().attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages, page_size, split_tokens))
+
+
+def decode_blasst_workspace_bytes(num_seqs, Hq, D, max_pages, page_size, split_tokens) -> int:
+    """Workspace of the tile-skip decode (scores, maxima and chunk partials)."""
+    return int(load_library().attn_decode_blasst_workspace_bytes(num_seqs, Hq, D, max_pages, page_size,
+                                                                 split_tokens))
 
 
 def decode_skip_mask_shape(num_seqs, Hkv, max_pages, page_size):
@@ -217,7 +248,7 @@ def decode_skip_mask_shape(num_seqs, Hkv, max_pages, page_size):
 
 
 def _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens, out, lse, workspace,
-            skip_mask, device_status, return_lse, stream, per_head=False):
+            skip_mask, device_status, return_lse, stream, per_head=False, skipped_tiles=None):
     _need(q, torch.bfloat16, 3, "q")
     _need(k_pages, torch.bfloat16, 4, "k_pages")
     _need(v_pages, torch.bfloat16, 4, "v_pages")
@@ -232,7 +263,10 @@ def _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens
     o = torch.empty_like(q) if out is None else out
     if lse is None and return_lse:
         lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device)
-    need = decode_workspace_bytes(N, Hq, D, max_pages, page_size, split_tokens)
+    skip_path = (lam > 0 or (skip_mask is not None and skip_mask is not False) or per_head
+                 or skipped_tiles is not None)
+    size_fn = decode_blasst_workspace_bytes if skip_path else decode_workspace_bytes
+    need = size_fn(N, Hq, D, max_pages, page_size, split_tokens)
     if need == 0:
         raise AttnError("invalid decode configuration", 1)
     if workspace is None:
@@ -247,7 +281,8 @@ def _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens
     st = fn(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), N, Hq, Hkv, D, page_size,
         max_pages, P, scale, lam, split_tokens, _ptr(o), _ptr(lse), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _ptr(mask), _ptr(device_status), _stream_handle(stream))
+        workspace.numel() * workspace.element_size(), _ptr(mask), _ptr(_counter(skipped_tiles, "skipped_tiles")),
+        _ptr(device_status), _stream_handle(stream))
     _check(st, "attn_decode_paged_blasst_heads" if per_head else "attn_decode_paged")
     return o, lse, mask
 
@@ -262,16 +297,20 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, split_t
 
 def decode_paged_blasst(q, k_pages, v_pages, block_table, seq_lens, lam: float, scale=None,
                         split_tokens: int = 1024, out=None, lse=None, workspace=None, skip_mask=True,
-                        device_status=None, return_lse=True, stream=None, rows_per_unit: str = "group"):
+                        device_status=None, return_lse=True, stream=None, rows_per_unit: str = "group",
+                        skipped_tiles=None):
     """Paged decode with the BLASST tile skip. Returns (o, lse, skip_mask).
 
     rows_per_unit="group": one decision per (sequence, KV head, tile) for the G
     query heads that share the KV head (mask [N, Hkv, tiles]); "head": one per
-    query head (mask [N, Hq, tiles])."""
+    query head (mask [N, Hq, tiles]). ``skipped_tiles`` (one-element int64
+    device tensor) receives the count of skipped decisions added to it. The
+    workspace, when given, must hold decode_blasst_workspace_bytes(...)."""
     if rows_per_unit not in ("group", "head"):
         raise AttnError("rows_per_unit must be 'group' or 'head'")
     return _decode(q, k_pages, v_pages, block_table, seq_lens, lam, scale, split_tokens, out, lse,
-                   workspace, skip_mask, device_status, return_lse, stream, per_head=rows_per_unit == "head")
+                   workspace, skip_mask, device_status, return_lse, stream, per_head=rows_per_unit == "head",
+                   skipped_tiles=skipped_tiles)
 
 
 def decode_paged_fp8(q, k_codes, v_codes, k_scale: float, v_scale: float, block_table, seq_lens, scale=None,
@@ -331,4 +370,19 @@ def decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale=None,
         block_table.shape[1], P, scale, 0.0, split_tokens, _ptr(o), _ptr(lse), None, _ptr(device_status),
         _stream_handle(stream))
     _check(st, "attn_decode_paged_noalloc")
+    return o, lse
+
+
+def debug_prefill_timeout(q, k, v, wait_limit_ns: int, withhold_step: int, causal: bool = True,
+                          scale: float | None = None, device_status=None, stream=None):
+    """TEST ONLY: a dense prefill whose pipeline waits give up after
+    ``wait_limit_ns`` and whose producer leaves out ring step ``withhold_step``
+    (-1: none). The output is undefined after a timeout; ``device_status`` then
+    holds ATTN_ERR_TIMEOUT (5). Returns (o, lse)."""
+    B, S, Hq, Hkv, D, o, lse = _prefill_args(q, k, v, None, None, True)
+    scale = default_scale(D) if scale is None else scale
+    st = load_library().attn_debug_prefill_timeout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, S,
+                                                   D, int(bool(causal)), scale, int(wait_limit_ns),
+                                                   int(withhold_step), _ptr(device_status), _stream_handle(stream))
+    _check(st, "attn_debug_prefill_timeout")
     return o, lse

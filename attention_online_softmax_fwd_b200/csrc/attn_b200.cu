@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_heads.cuh"
+#include "decode_blasst.cuh"
 #include "kv_append.cuh"
 #include "prefill.cuh"
 
@@ -119,19 +120,19 @@ int set_smem_once(int smem, int min_regs = 0) {
   return ATTN_OK;
 }
 
-// [B][S][H][D] bf16 tensor as a 4-D map {D, S, H, B}; box = 64 columns x 128 rows of one head.
-int encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+// [B][S][H][D] bf16 tensor as a 4-D map {D, S, H, B}; box = 64 columns x `rows` rows of one head.
+int encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int D, int rows = kPfRows) {
   const uint64_t dims[4] = {uint64_t(D), uint64_t(S), uint64_t(H), uint64_t(B)};
   const uint64_t strides[3] = {uint64_t(H) * D * 2, uint64_t(D) * 2, uint64_t(S) * H * D * 2};
-  const uint32_t box[4] = {64, uint32_t(kPfRows), 1, 1};
+  const uint32_t box[4] = {64, uint32_t(rows), 1, 1};
   return encode_map(map, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
 
 template <int D, bool CAUSAL, bool SKIP, bool PAGED = false>
-int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
-                   int sms, cudaStream_t stream) {
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tvh,
+                   const PrefillParams& p, int sms, cudaStream_t stream) {
   auto kernel = prefill_kernel<D, CAUSAL, SKIP, PAGED>;
   constexpr int smem = PrefillSmem<D>::kDynamic;
   // The kernel moves registers between warpgroups with setmaxnreg; the block's
@@ -141,22 +142,31 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
                                                                             kPfThreads))
     return st;
   const long long grid = p.num_items < sms ? p.num_items : sms;
-  kernel<<<dim3(unsigned(grid)), dim3(kPfThreads), smem, stream>>>(tq, tk, tv, p);
+  kernel<<<dim3(unsigned(grid)), dim3(kPfThreads), smem, stream>>>(tq, tk, tv, tvh, p);
   return launch_status();
 }
 
 template <int D, bool SKIP>
 int dispatch_prefill_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const PrefillParams& p, int sms, cudaStream_t stream) {
-  return causal ? launch_prefill<D, true, SKIP>(tq, tk, tv, p, sms, stream)
-                : launch_prefill<D, false, SKIP>(tq, tk, tv, p, sms, stream);
+                            const CUtensorMap& tvh, const PrefillParams& p, int sms, cudaStream_t stream) {
+  return causal ? launch_prefill<D, true, SKIP>(tq, tk, tv, tvh, p, sms, stream)
+                : launch_prefill<D, false, SKIP>(tq, tk, tv, tvh, p, sms, stream);
 }
 
+// Pipeline settings that only the test entry point changes.
+struct PrefillDebug {
+  unsigned long long wait_ns = kWaitLimitNs;
+  int withhold_step = -1;
+};
+
 int prefill_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S,
-                 int D, int causal, float scale, float lambda, uint8_t* skip_mask, int* device_status,
-                 void* stream, bool blasst) {
+                 int D, int causal, float scale, float lambda, uint8_t* skip_mask,
+                 unsigned long long* skipped_tiles, int* device_status, void* stream, bool blasst,
+                 const PrefillDebug& dbg = PrefillDebug()) {
   if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(skipped_tiles) & 7u))
+    return ATTN_ERR_INVALID_ARG;
   if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
@@ -169,7 +179,10 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.skip_mask = skip_mask;
+  p.skipped_tiles = skipped_tiles;
   p.status = device_status;
+  p.wait_ns = dbg.wait_ns;
+  p.withhold_step = dbg.withhold_step;
   p.B = B; p.S = S; p.Hq = Hq; p.Hkv = Hkv;
   p.n_qblocks = (S + 2 * kPfRows - 1) / (2 * kPfRows);
   p.n_qt = (S + kPfRows - 1) / kPfRows;
@@ -180,17 +193,19 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.scale_log2 = scale * 1.4426950408889634f;
   p.log2_lambda = lambda > 0.f ? std::log2(lambda) : -INFINITY;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tvh;
   if (int st = encode_bshd(&tq, q, B, S, Hq, D)) return st;
   if (int st = encode_bshd(&tk, k, B, S, Hkv, D)) return st;
   if (int st = encode_bshd(&tv, v, B, S, Hkv, D)) return st;
+  if (int st = encode_bshd(&tvh, v, B, S, Hkv, D, kPfKeys / 2)) return st;   // one 64-key half per box
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool use_skip = blasst && (lambda > 0.f || skip_mask != nullptr);  // the mask needs the decision path
+  // the mask and the count need the decision path
+  const bool use_skip = blasst && (lambda > 0.f || skip_mask != nullptr || skipped_tiles != nullptr);
   if (D == 128)
-    return use_skip ? dispatch_prefill_causal<128, true>(causal != 0, tq, tk, tv, p, sms, s)
-                    : dispatch_prefill_causal<128, false>(causal != 0, tq, tk, tv, p, sms, s);
-  return use_skip ? dispatch_prefill_causal<64, true>(causal != 0, tq, tk, tv, p, sms, s)
-                  : dispatch_prefill_causal<64, false>(causal != 0, tq, tk, tv, p, sms, s);
+    return use_skip ? dispatch_prefill_causal<128, true>(causal != 0, tq, tk, tv, tvh, p, sms, s)
+                    : dispatch_prefill_causal<128, false>(causal != 0, tq, tk, tv, tvh, p, sms, s);
+  return use_skip ? dispatch_prefill_causal<64, true>(causal != 0, tq, tk, tv, tvh, p, sms, s)
+                  : dispatch_prefill_causal<64, false>(causal != 0, tq, tk, tv, tvh, p, sms, s);
 }
 
 // Page pool [P][page_size][Hkv][D] as a 4-D map {D, Hkv, page_size, P}; box =
@@ -214,6 +229,72 @@ bool valid_page_size(int ps) { return ps == 16 || ps == 32 || ps == 64 || ps == 
 long long max_splits_of(int max_pages, int page_size, int split_tokens) {
   const long long cap = (long long)max_pages * page_size;
   return (cap + split_tokens - 1) / split_tokens;
+}
+
+// a * b into *out; false when the product does not fit a size_t
+bool mul_size(size_t a, size_t b, size_t* out) { return !__builtin_mul_overflow(a, b, out); }
+bool add_size(size_t a, size_t b, size_t* out) { return !__builtin_add_overflow(a, b, out); }
+
+// Bytes of the decode workspace [header][partial O][partial log2-sum-exp] for `slots`
+// (sequence, split) pairs; 0 when a size overflows. *o_bytes receives the partial-O bytes.
+size_t decode_ws_bytes(size_t slots, size_t Hq, size_t D, size_t* o_bytes) {
+  size_t rows = 0, ob = 0, lb = 0, total = 0;
+  if (!mul_size(slots, Hq, &rows) || !mul_size(rows, D * sizeof(float), &ob) || !mul_size(rows, sizeof(float), &lb))
+    return 0;
+  if (!add_size(ob, 255, &total)) return 0;
+  const size_t ob_aligned = total / 256 * 256;
+  if (!add_size(kWsHeader, ob_aligned, &total) || !add_size(total, lb, &total)) return 0;
+  if (o_bytes) *o_bytes = ob;
+  return total;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+// Workspace of the two-pass tile-skip decode, every part 256-byte aligned:
+//   [header: two work-ticket counters][partial O [N][max_chunks][Hq][D]][partial lse [N][max_chunks][Hq]]
+//   [scores [N][Hq][tok64]][tile maxima [N][Hq][max_tiles]][chunk maxima [N][Hq][max_chunks]]
+// A work item covers chunk_tokens tokens: the largest of 256, 192, 128, 64 that divides split_tokens (so
+// no chunk straddles a decision split), halved down to 64 while the batch gives fewer than 8192
+// (sequence, query head, chunk) triples, so that a few long sequences still fill the GPU.
+struct BlasstLayout {
+  int chunk = 0, max_chunks = 0, max_tiles = 0, tok64 = 0;
+  size_t o_off = 0, lse_off = 0, s_off = 0, tmax_off = 0, cmax_off = 0, total = 0;
+};
+
+bool blasst_layout(int num_seqs, int Hq, int D, int max_pages, int page_size, int split_tokens, BlasstLayout* L) {
+  if (num_seqs < 1 || Hq < 1 || (D != 64 && D != 128) || max_pages < 1 || !valid_page_size(page_size) ||
+      split_tokens < 64 || split_tokens % 64 != 0)
+    return false;
+  const long long cap = (long long)max_pages * page_size;
+  if (cap > (1ll << 30)) return false;
+  int C = 64;
+  for (int c : {256, 192, 128}) {
+    if (split_tokens % c == 0) { C = c; break; }
+  }
+  while (C % 128 == 0 && (long long)num_seqs * Hq * ((cap + C - 1) / C) < 8192) C /= 2;
+  L->chunk = C;
+  L->max_chunks = int((cap + C - 1) / C);
+  L->max_tiles = int((cap + 63) / 64);
+  L->tok64 = L->max_tiles * 64;
+  const size_t rows = size_t(num_seqs) * size_t(Hq);
+  size_t sz[5];
+  if (!mul_size(rows, size_t(L->max_chunks) * D * sizeof(float), &sz[0]) ||
+      !mul_size(rows, size_t(L->max_chunks) * sizeof(float), &sz[1]) ||
+      !mul_size(rows, size_t(L->tok64) * sizeof(float), &sz[2]) ||
+      !mul_size(rows, size_t(L->max_tiles) * sizeof(float), &sz[3]) ||
+      !mul_size(rows, size_t(L->max_chunks) * sizeof(float), &sz[4]))
+    return false;
+  size_t off = kWsHeader;
+  size_t* offs[5] = {&L->o_off, &L->lse_off, &L->s_off, &L->tmax_off, &L->cmax_off};
+  for (int i = 0; i < 5; ++i) {
+    *offs[i] = off;
+    size_t end = 0;
+    if (!add_size(off, sz[i], &end) || !add_size(end, 255, &end)) return false;
+    off = end / 256 * 256;
+  }
+  L->total = off;
+  return true;
 }
 
 // One CTA per (sequence, query head); a no-op for sequences of one split. Launched
@@ -291,6 +372,61 @@ int dispatch_decode_heads(int G, int hg, const CUtensorMap& tk, const CUtensorMa
   }
 }
 
+// Two-pass tile-skip decode: pass 1 (scores and maxima), pass 2 (decisions, kept V, P V) as a programmatic
+// dependent of pass 1, then the merge of the chunk partials as a programmatic dependent of pass 2.
+template <int D, int G, int HG, bool PER_HEAD>
+int launch_blasst(const CUtensorMap& tk, const CUtensorMap& tvg, const CUtensorMap& tvh, const DecodeParams& p,
+                  int* tickets, int sms, cudaStream_t stream) {
+  using L1 = BlScoresSmem<D, G, HG>;
+  using L2 = BlPvSmem<D, G, HG>;
+  if (int st = set_smem_once<decode_scores_kernel<D, G, HG>>(L1::kDynamic)) return st;
+  if (int st = set_smem_once<decode_pv_kernel<D, G, HG, PER_HEAD>>(L2::kDynamic)) return st;
+  const long long items = (long long)p.max_chunks * p.num_seqs * (p.Hkv / HG);
+  const long long slots1 = (long long)sms * L1::kBlocks, slots2 = (long long)sms * L2::kBlocks;
+  decode_scores_kernel<D, G, HG><<<dim3(unsigned(items < slots1 ? items : slots1)), dim3((HG + 1) * 32),
+                                   L1::kDynamic, stream>>>(tk, p, tickets);
+  if (int st = launch_status()) return st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(items < slots2 ? items : slots2));
+  cfg.blockDim = dim3((HG + 1) * 32);
+  cfg.dynamicSmemBytes = L2::kDynamic;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, decode_pv_kernel<D, G, HG, PER_HEAD>, tvg, tvh, p, tickets + 1) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (int st = launch_status()) return st;
+  DecodeParams pm = p;          // the merge combines chunk partials
+  pm.split_tokens = p.chunk_tokens;
+  pm.max_splits = p.max_chunks;
+  return launch_merge<D>(pm, stream);
+}
+
+template <int D, int HG, bool PER_HEAD>
+int dispatch_blasst_g(int G, const CUtensorMap& tk, const CUtensorMap& tvg, const CUtensorMap& tvh,
+                      const DecodeParams& p, int* tickets, int sms, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_blasst<D, 1, HG, PER_HEAD>(tk, tvg, tvh, p, tickets, sms, s);
+    case 2: return launch_blasst<D, 2, HG, PER_HEAD>(tk, tvg, tvh, p, tickets, sms, s);
+    case 4: return launch_blasst<D, 4, HG, PER_HEAD>(tk, tvg, tvh, p, tickets, sms, s);
+    case 8: return launch_blasst<D, 8, HG, PER_HEAD>(tk, tvg, tvh, p, tickets, sms, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+template <int D>
+int dispatch_blasst(int G, int hg, bool per_head, const CUtensorMap& tk, const CUtensorMap& tvg,
+                    const CUtensorMap& tvh, const DecodeParams& p, int* tickets, int sms, cudaStream_t s) {
+  if (hg == 4)
+    return per_head ? dispatch_blasst_g<D, 4, true>(G, tk, tvg, tvh, p, tickets, sms, s)
+                    : dispatch_blasst_g<D, 4, false>(G, tk, tvg, tvh, p, tickets, sms, s);
+  return per_head ? dispatch_blasst_g<D, 1, true>(G, tk, tvg, tvh, p, tickets, sms, s)
+                  : dispatch_blasst_g<D, 1, false>(G, tk, tvg, tvh, p, tickets, sms, s);
+}
+
 // FP8 cache (D = 128): groups of 4 KV heads for G <= 8; G = 16 takes groups of hg (8 or 4)
 int dispatch_decode_heads_fp8(int G, int hg, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                               int* ctr, int sms, cudaStream_t s) {
@@ -321,18 +457,38 @@ const char* attn_status_string(int status) {
   }
 }
 
-int attn_abi_version(void) { return 1; }
+int attn_abi_version(void) { return 2; }
 
 int attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S,
                  int D, int causal, float scale, void* stream) {
-  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, 0.f, nullptr, nullptr, stream, false);
+  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, 0.f, nullptr, nullptr, nullptr, stream,
+                      false);
 }
 
 int attn_prefill_blasst(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                         int S, int D, int causal, float scale, float lambda, uint8_t* skip_mask,
-                        int* device_status, void* stream) {
-  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, lambda, skip_mask, device_status, stream,
-                      true);
+                        unsigned long long* skipped_tiles, int* device_status, void* stream) {
+  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, lambda, skip_mask, skipped_tiles,
+                      device_status, stream, true);
+}
+
+int attn_debug_prefill_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                               int Hkv, int S, int D, int causal, float scale, unsigned long long wait_limit_ns,
+                               int withhold_step, int* device_status, void* stream) {
+  if (wait_limit_ns < 1000ull || wait_limit_ns > kWaitLimitNs) return ATTN_ERR_INVALID_ARG;
+  PrefillDebug dbg;
+  dbg.wait_ns = wait_limit_ns;
+  dbg.withhold_step = withhold_step < 0 ? -1 : withhold_step;
+  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, 0.f, nullptr, nullptr, device_status,
+                      stream, false, dbg);
+}
+
+int attn_set_library_status(int enable) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int on = enable ? 1 : 0;
+  if (cudaMemcpyToSymbol(g_library_status_on, &on, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
 }
 
 int attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
@@ -372,14 +528,16 @@ int attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages, 
   p.max_pages = max_pages_per_seq;
   p.num_pages = num_pages;
   p.page_size = page_size;
+  p.wait_ns = kWaitLimitNs;
+  p.withhold_step = -1;
 
   CUtensorMap tq, tk, tv;
   if (int st = encode_bshd(&tq, q, B, Sq, Hq, D)) return st;
   if (int st = encode_pool16(&tk, k_pages, num_pages, page_size, Hkv, D)) return st;
   if (int st = encode_pool16(&tv, v_pages, num_pages, page_size, Hkv, D)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return D == 128 ? launch_prefill<128, true, false, true>(tq, tk, tv, p, sms, s)
-                  : launch_prefill<64, true, false, true>(tq, tk, tv, p, sms, s);
+  return D == 128 ? launch_prefill<128, true, false, true>(tq, tk, tv, tv, p, sms, s)
+                  : launch_prefill<64, true, false, true>(tq, tk, tv, tv, p, sms, s);
 }
 
 size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq, int page_size,
@@ -388,20 +546,30 @@ size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_pe
       split_tokens < 64 || split_tokens % 64 != 0)
     return 0;
   const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
-  const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
-  const size_t o_bytes_aligned = (o_bytes + 255) / 256 * 256;
-  return kWsHeader + o_bytes_aligned + size_t(num_seqs) * ms * Hq * sizeof(float);
+  size_t slots = 0;
+  if (!mul_size(size_t(num_seqs), size_t(ms), &slots)) return 0;
+  return decode_ws_bytes(slots, size_t(Hq), size_t(D), nullptr);
+}
+
+size_t attn_decode_blasst_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq, int page_size,
+                                          int split_tokens) {
+  BlasstLayout L;
+  if (!blasst_layout(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens, &L)) return 0;
+  const size_t dense = attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens);
+  return dense > L.total ? dense : L.total;
 }
 
 static int decode_impl(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
                        const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
                        int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens, void* o,
                        float* lse, void* workspace, size_t workspace_bytes, uint8_t* skip_mask,
-                       int* device_status, void* stream, bool per_head) {
+                       unsigned long long* skipped_tiles, int* device_status, void* stream, bool per_head) {
   if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace))
     return ATTN_ERR_INVALID_ARG;
+  if (!aligned4(block_table) || !aligned4(seq_lens) || !aligned4(lse)) return ATTN_ERR_INVALID_ARG;
   if (num_seqs < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if ((long long)num_seqs * Hq > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;   // one merge CTA per (sequence, head)
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   if (!valid_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
   if (split_tokens < 64 || split_tokens % 64 != 0) return ATTN_ERR_INVALID_ARG;
@@ -410,12 +578,18 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
   if ((long long)max_pages_per_seq * page_size > (1ll << 30)) return ATTN_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return ATTN_ERR_UNSUPPORTED;
-  const size_t need = attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens);
+  if (!aligned8(skipped_tiles)) return ATTN_ERR_INVALID_ARG;
+  const bool use_skip = lambda > 0.f || skip_mask != nullptr || skipped_tiles != nullptr || per_head;
+  const size_t need = use_skip ? attn_decode_blasst_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size,
+                                                                    split_tokens)
+                               : attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size,
+                                                             split_tokens);
   if (need == 0 || workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
   int sms = 0;
   if (int st = current_device(&sms)) return st;
 
   DecodeParams p{};
+  p.skipped_tiles = skipped_tiles;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.block_table = block_table;
   p.seq_lens = seq_lens;
@@ -424,7 +598,8 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
   const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
   int* ticket_counter = static_cast<int*>(workspace);
   p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader);
-  const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
+  size_t o_bytes = 0;
+  decode_ws_bytes(size_t(num_seqs) * size_t(ms), size_t(Hq), size_t(D), &o_bytes);   // checked above
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader + (o_bytes + 255) / 256 * 256);
   p.skip_mask = skip_mask;
   p.status = device_status;
@@ -448,13 +623,36 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
   if (int st = encode_map5(&tk, k_pages, dims, strides, box)) return st;
   if (int st = encode_map5(&tv, v_pages, dims, strides, box)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool use_skip = lambda > 0.f || skip_mask != nullptr || per_head;
   const int hg = G <= 8 ? (Hkv % 4 == 0 ? 4 : 0) : (Hkv % 8 == 0 ? 8 : (Hkv == 4 ? 4 : 0));
+  // {64 columns, token, 64-column half, head, page}: a head's 16 tokens land as [half][token][64]
+  const uint64_t hdims[5] = {64, uint64_t(page_size), uint64_t(D / 64), uint64_t(Hkv), uint64_t(num_pages)};
+  const uint64_t hstrides[4] = {uint64_t(Hkv) * D * 2, 128, uint64_t(D) * 2, uint64_t(page_size) * Hkv * D * 2};
+  if (use_skip && G <= 8) {
+    // two passes over groups of 4 KV heads (of 1 when Hkv is not a multiple of 4)
+    const int bhg = Hkv % 4 == 0 ? 4 : 1;
+    BlasstLayout BL;
+    blasst_layout(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens, &BL);   // checked above
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.ws_o = reinterpret_cast<float*>(ws + BL.o_off);
+    p.ws_lse = reinterpret_cast<float*>(ws + BL.lse_off);
+    p.ws_s = reinterpret_cast<float*>(ws + BL.s_off);
+    p.ws_tmax = reinterpret_cast<float*>(ws + BL.tmax_off);
+    p.ws_cmax = reinterpret_cast<float*>(ws + BL.cmax_off);
+    p.chunk_tokens = BL.chunk;
+    p.max_chunks = BL.max_chunks;
+    p.tok64 = BL.tok64;
+    const uint32_t gbox[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), uint32_t(bhg), 1};
+    const uint32_t box1[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), 1, 1};
+    CUtensorMap bk, bvg, bvh;
+    if (int st = encode_map5(&bk, k_pages, hdims, hstrides, gbox)) return st;
+    if (int st = encode_map5(&bvg, v_pages, hdims, hstrides, gbox)) return st;
+    if (int st = encode_map5(&bvh, v_pages, hdims, hstrides, box1)) return st;
+    if (cudaMemsetAsync(ticket_counter, 0, 2 * sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (D == 128) return dispatch_blasst<128>(G, bhg, per_head, bk, bvg, bvh, p, ticket_counter, sms, s);
+    return dispatch_blasst<64>(G, bhg, per_head, bk, bvg, bvh, p, ticket_counter, sms, s);
+  }
   if (!use_skip && hg > 0) {
     // dense: one item per group of hg KV heads, 16-token stages covering all of them
-    // {64 columns, token, 64-column half, head, page}: a head's 16 tokens land as [half][token][64]
-    const uint64_t hdims[5] = {64, uint64_t(page_size), uint64_t(D / 64), uint64_t(Hkv), uint64_t(num_pages)};
-    const uint64_t hstrides[4] = {uint64_t(Hkv) * D * 2, 128, uint64_t(D) * 2, uint64_t(page_size) * Hkv * D * 2};
     const uint32_t hbox[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), uint32_t(hg), 1};
     CUtensorMap hk, hv;
     if (int st = encode_map5(&hk, k_pages, hdims, hstrides, hbox)) return st;
@@ -504,21 +702,22 @@ int attn_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_
 int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
                       const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
                       int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens, void* o,
-                      float* lse, void* workspace, size_t workspace_bytes, uint8_t* skip_mask, int* device_status,
-                      void* stream) {
+                      float* lse, void* workspace, size_t workspace_bytes, uint8_t* skip_mask,
+                      unsigned long long* skipped_tiles, int* device_status, void* stream) {
   return decode_impl(q, k_pages, v_pages, block_table, seq_lens, num_seqs, Hq, Hkv, D, page_size,
                      max_pages_per_seq, num_pages, scale, lambda, split_tokens, o, lse, workspace, workspace_bytes,
-                     skip_mask, device_status, stream, false);
+                     skip_mask, skipped_tiles, device_status, stream, false);
 }
 
 int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const void* v_pages,
                                    const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int Hq,
                                    int Hkv, int D, int page_size, int max_pages_per_seq, int num_pages, float scale,
                                    float lambda, int split_tokens, void* o, float* lse, void* workspace,
-                                   size_t workspace_bytes, uint8_t* skip_mask, int* device_status, void* stream) {
+                                   size_t workspace_bytes, uint8_t* skip_mask, unsigned long long* skipped_tiles,
+                                   int* device_status, void* stream) {
   return decode_impl(q, k_pages, v_pages, block_table, seq_lens, num_seqs, Hq, Hkv, D, page_size,
                      max_pages_per_seq, num_pages, scale, lambda, split_tokens, o, lse, workspace, workspace_bytes,
-                     skip_mask, device_status, stream, true);
+                     skip_mask, skipped_tiles, device_status, stream, true);
 }
 
 int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_codes, float k_scale, float v_scale,
@@ -529,9 +728,9 @@ int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_code
   if (!q || !k_codes || !v_codes || !block_table || !seq_lens || !o || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(o) || !aligned16(workspace))
     return ATTN_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
-    return ATTN_ERR_INVALID_ARG;
+  if (!aligned4(block_table) || !aligned4(seq_lens) || !aligned4(lse)) return ATTN_ERR_INVALID_ARG;
   if (num_seqs < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if ((long long)num_seqs * Hq > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;   // one merge CTA per (sequence, head)
   if (!valid_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
   if (split_tokens < 64 || split_tokens % 64 != 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
@@ -560,7 +759,8 @@ int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_code
   const long long ms = max_splits_of(max_pages_per_seq, page_size, split_tokens);
   int* ticket_counter = static_cast<int*>(workspace);
   p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader);
-  const size_t o_bytes = size_t(num_seqs) * ms * Hq * D * sizeof(float);
+  size_t o_bytes = 0;
+  decode_ws_bytes(size_t(num_seqs) * size_t(ms), size_t(Hq), size_t(D), &o_bytes);   // checked above
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeader + (o_bytes + 255) / 256 * 256);
   p.status = device_status;
   p.num_seqs = num_seqs; p.Hq = Hq; p.Hkv = Hkv;
@@ -625,13 +825,17 @@ int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_
                               const int32_t* seq_lens, int num_seqs, int Hq, int Hkv, int D, int page_size,
                               int max_pages_per_seq, int num_pages, float scale, float lambda, int split_tokens,
                               void* o, float* lse, uint8_t* skip_mask, int* device_status, void* stream) {
-  const size_t need = attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size, split_tokens);
+  const bool skip_path = lambda > 0.f || skip_mask != nullptr;
+  const size_t need = skip_path ? attn_decode_blasst_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size,
+                                                                     split_tokens)
+                                : attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size,
+                                                              split_tokens);
   if (need == 0 || need > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_INVALID_ARG;
   void* scratch = nullptr;
   if (int st = noalloc_scratch(&scratch)) return st;
   return attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_seqs, Hq, Hkv, D, page_size,
                            max_pages_per_seq, num_pages, scale, lambda, split_tokens, o, lse, scratch,
-                           ATTN_NOALLOC_SCRATCH_BYTES, skip_mask, device_status, stream);
+                           ATTN_NOALLOC_SCRATCH_BYTES, skip_mask, nullptr, device_status, stream);
 }
 
 int attn_read_device_status(int* status_out, int clear) {

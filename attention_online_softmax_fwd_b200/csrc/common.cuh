@@ -14,14 +14,18 @@
 
 namespace attn {
 
-// Library-wide device status word (the larger code wins).
+// Library-wide device status word (the larger code wins). Kernels record into
+// it only after the caller has switched it on for the device
+// (attn_set_library_status); by default every error goes to the caller's own
+// status word alone and the library keeps no state that calls share.
 __device__ int g_device_status = ATTN_OK;
+__device__ int g_library_status_on = 0;
 
 // A pipeline wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ void raise_status(int* user_status, int code) {
-  atomicMax(&g_device_status, code);
+  if (g_library_status_on) atomicMax(&g_device_status, code);
   if (user_status) atomicMax(user_status, code);
 }
 
@@ -76,14 +80,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // the CTA was told to abort or the wait ran out of time (then the abort flag
 // is raised so that every other role of the CTA stops too).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* user_status) {
+                                          int* user_status, unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         raise_status(user_status, ATTN_ERR_TIMEOUT);
         return false;
@@ -414,7 +418,7 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
 
 // 2^x for a pair, on the FMA pipe: x = n + f with n = round(x) (obtained by
 // adding 1.5 * 2^23, which leaves n in the low mantissa bits), f in [-1/2, 1/2];
-// 2^f by a cubic fitted by fit_exp2_poly.py (max relative error 7.7e-5);
+// 2^f by a cubic fitted by tests/exp2_poly_fit.py (max relative error 7.7e-5);
 // 2^n applied by adding n to the exponent field. Inputs are clamped to
 // [-126, 64], so masked (-inf) entries come out as ~1e-38.
 __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {

@@ -48,6 +48,13 @@ struct DecodeParams {
   float v_scale;      // FP8 cache: V = v_scale * code (the K scale is folded into scale_log2)
   int per_head;       // tile skip decided for each query head alone, not for the KV head's group
   long long num_items;
+  // two-pass tile-skip decode (decode_blasst.cuh); the work items are chunks of
+  // chunk_tokens tokens (a divisor of split_tokens), the decision units are splits
+  float* ws_s;        // scaled scores (log2 units) [N][Hkv / HG][tok64][HG][G]
+  float* ws_tmax;     // row maxima of every 64-token tile [N][Hq][max_tiles]
+  float* ws_cmax;     // row maxima of every chunk [N][Hq][max_chunks]
+  unsigned long long* skipped_tiles;   // count of skipped decisions, or null
+  int chunk_tokens, max_chunks, tok64;
 };
 
 constexpr int kDecTile = 64;          // tokens per tile (= BLASST decision tile)
@@ -411,6 +418,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 p.skip_mask[(size_t(seq) * p.Hq + kvh * G + row) * p.max_tiles + t0 / kDecTile] = skip_r[rr] ? 1 : 0;
             }
           }
+          if (p.skipped_tiles && warp == 0) {
+            const int n = __popc(__ballot_sync(0xffffffffu, tq == 0 && row0_valid && skip_r[0])) +
+                          __popc(__ballot_sync(0xffffffffu, tq == 0 && row1_valid && skip_r[1]));
+            if (lane == 0 && n) atomicAdd(p.skipped_tiles, (unsigned long long)n);
+          }
         } else {
           skip_r[0] = skip_r[1] = false;
           if (!skip) {
@@ -419,6 +431,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           }
           if (p.skip_mask && warp == 0 && lane == 0)
             p.skip_mask[(size_t(seq) * p.Hkv + kvh) * p.max_tiles + t0 / kDecTile] = skip ? 1 : 0;
+          if (p.skipped_tiles && warp == 0 && lane == 0 && skip) atomicAdd(p.skipped_tiles, 1ull);
         }
       }
 

@@ -48,6 +48,9 @@ struct PrefillParams {
   const __nv_bfloat16* k_pool;   // [num_pages][page_size][Hkv][D]
   const __nv_bfloat16* v_pool;
   int max_pages, num_pages, page_size;
+  unsigned long long* skipped_tiles;   // tile skip: count of skipped (query tile, 64-key tile) decisions, or null
+  unsigned long long wait_ns;          // pipeline wait limit (kWaitLimitNs unless a test shortens it)
+  int withhold_step;                   // test only: the producer leaves out this ring step (-1: none)
 };
 
 constexpr int kPfRows = 128;     // rows per query tile
@@ -137,14 +140,14 @@ __device__ __forceinline__ bool pf_votes_all_in(const int4& w, int tag) {
 // Kept out of line: it runs only when a vote is late, and inlined it would
 // crowd the registers of the softmax loop.
 __device__ __forceinline__ int pf_tile_decision_wait(const volatile int* words, int tag, volatile int* abort_flag,
-                                                  int* user_status) {
+                                                  int* user_status, unsigned long long limit_ns) {
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     const int4 w = pf_votes_v4(words);
     if (pf_votes_all_in(w, tag)) return w.x & w.y & w.z & w.w & 3;
     if ((i & 31u) == 0) {
       if (*abort_flag) return -1;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         raise_status(user_status, ATTN_ERR_TIMEOUT);
         return -1;
@@ -154,10 +157,63 @@ __device__ __forceinline__ int pf_tile_decision_wait(const volatile int* words, 
 }
 
 __device__ __forceinline__ int pf_tile_decision(const volatile int* words, int tag, volatile int* abort_flag,
-                                                int* user_status) {
+                                                int* user_status, unsigned long long limit_ns) {
   const int4 w = pf_votes_v4(words);
   if (pf_votes_all_in(w, tag)) return w.x & w.y & w.z & w.w & 3;
-  return pf_tile_decision_wait(words, tag, abort_flag, user_status);
+  return pf_tile_decision_wait(words, tag, abort_flag, user_status, limit_ns);
+}
+
+// The V load of a K/V tile shared by the two query tiles: the halves that both
+// drop (bit h: 64-key half h), once both warpgroups' votes are in; -1 on
+// timeout. tag_x is the tile's vote sequence number in warpgroup x, 0 when query
+// tile x does not visit the tile (it then drops both halves).
+__device__ __forceinline__ int pf_dropped_by_both(const volatile int* votes, int tag0, int tag1,
+                                                  volatile int* abort_flag, int* user_status,
+                                                  unsigned long long limit_ns) {
+  unsigned long long t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    int d = 3;
+    bool in = true;
+    if (tag0) {
+      const int4 w = pf_votes_v4(votes + (tag0 & 3) * 4);
+      in = in && pf_votes_all_in(w, tag0);
+      d &= w.x & w.y & w.z & w.w;
+    }
+    if (tag1) {
+      const int4 w = pf_votes_v4(votes + 16 + (tag1 & 3) * 4);
+      in = in && pf_votes_all_in(w, tag1);
+      d &= w.x & w.y & w.z & w.w;
+    }
+    if (in) return d & 3;
+    if (i == 0) {
+      t0 = global_timer_ns();
+    } else if ((i & 31u) == 0) {
+      if (*abort_flag) return -1;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        raise_status(user_status, ATTN_ERR_TIMEOUT);
+        return -1;
+      }
+    }
+  }
+}
+
+// The order of one item's K and V tiles in the ring: K_0 .. K_{L-1}, then V_j and
+// K_{j+L} in turn, then the last V tiles. With L = 2 each K_{j+1} is loaded just
+// before V_j; the tile skip uses L = 3, so that the skip decision on tile j is in
+// before V_j is due and a dropped tile's V need not be loaded.
+template <int L>
+__device__ __forceinline__ void pf_ring_step(int step, int n, bool& is_k, int& tile) {
+  const int a = n < L ? n : L;
+  if (step < a) { is_k = true; tile = step; return; }
+  const int st = step - a, m = n - a;
+  if (st < 2 * m) {
+    is_k = (st & 1) != 0;
+    tile = (st >> 1) + (is_k ? L : 0);
+    return;
+  }
+  is_k = false;
+  tile = m + (st - 2 * m);
 }
 
 // Row-sum pairs (exact, as rounded for P V), added and scaled without contraction.
@@ -269,18 +325,36 @@ __device__ __forceinline__ void pf_write_skip_mask(const PrefillParams& p, int b
   }
 }
 
+// The visited 64-key tiles among the two of K/V tile jt that decision d drops.
+template <bool CAUSAL>
+__device__ __forceinline__ int pf_count_skipped(const PrefillParams& p, int jt, int last_row, int decision) {
+  int n = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k64 = jt * kPfKeys + h * 64;
+    const bool visited = k64 < p.S && (!CAUSAL || k64 <= last_row);
+    n += (visited && ((decision >> h) & 1)) ? 1 : 0;
+  }
+  return n;
+}
+
 // PAGED: chunked prefill. Query row i of sequence b sits at position
 // L_b - S + i (L_b = seq_lens[b]) and sees cached keys 0 .. L_b - S + i; the K
 // and V tiles are gathered from the page pool through the block table, one
 // box of 16 keys at a time (pf_load_paged_tile; tm_k / tm_v then map the pools as
 // {D, Hkv, page_size, P} with 16-slot boxes).
+// SKIP: tm_vh maps V with boxes of 64 rows (one 64-key half of a tile), so that
+// the producer loads only the halves that one of the two query tiles keeps.
 template <int D, bool CAUSAL, bool SKIP, bool PAGED = false>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_vh,
+                   const PrefillParams p) {
   using L = PrefillSmem<D>;
   constexpr int NS = L::kStages;
   constexpr int kTmemCols = 512;
+  constexpr int kLead = SKIP ? 3 : 2;   // K tiles loaded before the first V (pf_ring_step)
+
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -383,7 +457,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int x = 0; x < 2; ++x) {
           if ((x == 0 ? rows0 : rows1) == 0 || !ok) continue;
           int w = 1;
-          if (lane == 0) w = mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status) ? 1 : 0;
+          if (lane == 0)
+            w = mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status, p.wait_ns) ? 1 : 0;
           if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; continue; }
           qe_bits ^= 1u << x;
           if (lane == 0) {
@@ -401,17 +476,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int pre = pf_page_entry(p, b, 0, g, n_keys);
         int entry_even = p.num_pages, entry_odd = p.num_pages;   // of the last K tiles with even / odd index
         for (int step = 0; step < 2 * n && ok; ++step) {
-          const int j = (step - 1) / 2;
-          const bool is_k = step == 0 || (step % 2 == 1 && j + 1 < n);
-          const int key0 = step == 0 ? 0 : (is_k ? (j + 1) * kPfKeys : (step % 2 == 1 ? j : step / 2 - 1) * kPfKeys);
-          const int tile = key0 / kPfKeys;
+          bool is_k;
+          int tile;
+          pf_ring_step<kLead>(step, n, is_k, tile);
+          const int key0 = tile * kPfKeys;
           if (is_k) {
             if (tile & 1) entry_odd = pre; else entry_even = pre;
             pre = pf_page_entry(p, b, tile + 1, g, n_keys);
           }
           const int entry = (tile & 1) ? entry_odd : entry_even;
           int w = 1;
-          if (lane == 0) w = mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status) ? 1 : 0;
+          if (lane == 0) w = mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status, p.wait_ns) ? 1 : 0;
           if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
           if (lane == 0) mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
           if (lane < kPfKeys / 16)
@@ -438,6 +513,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         uint32_t phase = 0;
         uint32_t qe_bits = 3u;
         uint32_t pend_mask = 0, pend_ph = 0;
+        int vseq[2] = {0, 0};   // SKIP: the tiles each softmax warpgroup has voted on (its vote sequence)
+        int gstep = 0;          // ring steps of this CTA (for the test-only withheld step)
         bool ok = true;
         for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
           int qb, b, hq;
@@ -445,11 +522,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const int kvh = hq / (p.Hq / p.Hkv);
           const int off = seq_offset(b, false);
           const int rows0 = tile_rows(qb, 0), rows1 = tile_rows(qb, 1);
-          const int n = max(tile_nkv(qb, 0, rows0, off), tile_nkv(qb, 1, rows1, off));
+          const int nkv0 = tile_nkv(qb, 0, rows0, off), nkv1 = tile_nkv(qb, 1, rows1, off);
+          const int n = max(nkv0, nkv1);
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if ((x == 0 ? rows0 : rows1) == 0 || !ok) continue;
-            if (!mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status)) { ok = false; continue; }
+            if (!mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status, p.wait_ns)) {
+              ok = false;
+              continue;
+            }
             qe_bits ^= 1u << x;
             mbar_arrive_expect_tx(&bars[L::bQFull + x], L::kTileBytes);
 #pragma unroll
@@ -457,21 +538,50 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               tma_load_4d(smem + L::kQ + x * L::kTileBytes + c * L::kChunkBytes, &tm_q, &bars[L::bQFull + x],
                           c * 64, qb * 2 * kPfRows + x * kPfRows, hq, b);
           }
-          // K_0, then K_{j+1} before V_j: the order in which the MMA thread consumes them
+          // the order in which the MMA issuers consume the tiles (pf_ring_step)
           for (int step = 0; step < 2 * n && ok; ++step) {
-            // step 0: K_0; step 2j+1: K_{j+1} (or V_j when j is the last tile); step 2j+2: V_j
-            const int j = (step - 1) / 2;
-            const bool is_k = step == 0 || (step % 2 == 1 && j + 1 < n);
-            const int key0 = step == 0 ? 0 : (is_k ? (j + 1) * kPfKeys : (step % 2 == 1 ? j : step / 2 - 1) * kPfKeys);
-            if (!mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-            mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
-            const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+            bool is_k;
+            int tile;
+            pf_ring_step<kLead>(step, n, is_k, tile);
+            const int key0 = tile * kPfKeys;
+            int halves = 3;   // bit h: 64-key half h of the tile is loaded
+            if constexpr (SKIP) {
+              if (!is_k) {
+                // V_tile is loaded only for the halves that one of the two query tiles keeps; both
+                // softmax warpgroups have voted on the tile by now (K runs kLead tiles ahead)
+                const int tag0 = tile < nkv0 ? ++vseq[0] : 0;   // 0: this query tile does not visit it
+                const int tag1 = tile < nkv1 ? ++vseq[1] : 0;
+                const int dropped = pf_dropped_by_both(votes, tag0, tag1, abort_flag, p.status, p.wait_ns);
+                if (dropped < 0) { ok = false; break; }
+                halves = ~dropped & 3;
+              }
+            }
+            if (!mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            if (gstep++ != p.withhold_step) {
+              uint8_t* dst = smem + L::kRing + slot * L::kTileBytes;
+              if (halves == 3) {
+                mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
+                const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_4d(smem + L::kRing + slot * L::kTileBytes + c * L::kChunkBytes, tm, &bars[L::bKVFull + slot],
-                          c * 64, key0, kvh, b);
-            pend_mask |= 1u << slot;
-            pend_ph = (pend_ph & ~(1u << slot)) | (phase << slot);
+                for (int c = 0; c < D / 64; ++c)
+                  tma_load_4d(dst + c * L::kChunkBytes, tm, &bars[L::bKVFull + slot], c * 64, key0, kvh, b);
+              } else {
+                mbar_arrive_expect_tx(&bars[L::bKVFull + slot], uint32_t(__popc(halves)) * (L::kTileBytes / 2));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  if (!((halves >> h) & 1)) continue;
+#pragma unroll
+                  for (int c = 0; c < D / 64; ++c)
+                    tma_load_4d(dst + c * L::kChunkBytes + h * (L::kChunkBytes / 2), &tm_vh, &bars[L::bKVFull + slot],
+                                c * 64, key0 + 64 * h, kvh, b);
+                }
+              }
+              pend_mask |= 1u << slot;
+              pend_ph = (pend_ph & ~(1u << slot)) | (phase << slot);
+            }
             if (++slot == NS) { slot = 0; phase ^= 1u; }
           }
         }
@@ -507,24 +617,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const int n = max(tile_nkv(qb, 0, rows0, off), tile_nkv(qb, 1, rows1, off));
           const int nkv = tile_nkv(qb, x, x == 0 ? rows0 : rows1, off);
           if (nkv > 0) {
-            if (!mbar_wait(&bars[L::bQFull + x], qf_ph, abort_flag, p.status)) break;
+            if (!mbar_wait(&bars[L::bQFull + x], qf_ph, abort_flag, p.status, p.wait_ns)) break;
             qf_ph ^= 1u;
           }
           bool pv_started = false;  // a P V product was issued for this tile in this item
-          // ring uses of the item, in order: K_0, then K_{j+1} (if any) and V_j for each j
+          // ring uses of the item, in the producer's order (pf_ring_step)
           for (int step = 0; step < 2 * n && ok; ++step) {
-            const int j = (step - 1) / 2;
-            const bool is_k = step == 0 || (step % 2 == 1 && j + 1 < n);
-            const int tile = step == 0 ? 0 : (is_k ? j + 1 : (step % 2 == 1 ? j : step / 2 - 1));
+            bool is_k;
+            int tile;
+            pf_ring_step<kLead>(step, n, is_k, tile);
             const int cur = slot;
             const uint32_t cph = phase;
             if (++slot == NS) { slot = 0; phase ^= 1u; }
-            if (!mbar_wait(&bars[L::bKVFull + cur], cph, abort_flag, p.status)) { ok = false; break; }
+            if (!mbar_wait(&bars[L::bKVFull + cur], cph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             if (is_k && tile < nkv) {
               // S_x(tile) = Q_x K_tile^T, once the softmax has copied out S_x(tile - 1)
               if (qk_started) {
-                if (!mbar_wait(&bars[L::bSFree + x], sfree_ph, abort_flag, p.status)) { ok = false; break; }
+                if (!mbar_wait(&bars[L::bSFree + x], sfree_ph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 sfree_ph ^= 1u;
                 tc_fence_after();
               }
@@ -535,20 +645,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (tile + 1 == nkv) umma_commit(&bars[L::bQEmpty + x]);   // last Q K^T of this tile
             } else if (!is_k && tile < nkv) {
               // O_x += P_x(tile) V_tile
-              if (!mbar_wait(&bars[L::bPFull + x], pf_ph, abort_flag, p.status)) { ok = false; break; }
+              if (!mbar_wait(&bars[L::bPFull + x], pf_ph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
               pf_ph ^= 1u;
               tc_fence_after();
               int skip_halves = 0;
               if constexpr (SKIP) {
                 // every softmax warp voted before arriving on P_full
                 ++seq;
-                skip_halves = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, abort_flag, p.status);
+                skip_halves = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, abort_flag, p.status, p.wait_ns);
                 if (skip_halves < 0) { ok = false; break; }
               }
               if (skip_halves != 3) {
                 if (!pv_started) {
                   // first P V of this item: the previous item's epilogue must have read O_x
-                  if (!mbar_wait(&bars[L::bOEmpty + x], oe_ph, abort_flag, p.status)) { ok = false; break; }
+                  if (!mbar_wait(&bars[L::bOEmpty + x], oe_ph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                   oe_ph ^= 1u;
                   tc_fence_after();
                 }
@@ -579,6 +689,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // this thread's row of P (K-major, 128-byte swizzle, two 64-key chunks)
     uint8_t* prow = smem + L::kP + x * L::kPBytes + t * 128;
     const float neg_inf = -__int_as_float(0x7f800000);
+    // The softmax waits stop on their own limit only (the full one: the test entry point shortens the
+    // producer's and issuers' waits, which then give up first; these follow within the full limit).
     int own_timeout_only = 0;
     volatile int* no_abort = reinterpret_cast<volatile int*>(&own_timeout_only);
     uint32_t sf_ph = 0, pvd_ph = 0;
@@ -598,6 +710,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const bool row_valid = t < rows;
       const int last_row = row0 + rows - 1;
       float m_ref = neg_inf, m_true = neg_inf;
+      int n_skipped = 0;   // SKIP, thread 0: dropped visited 64-key tiles of this query tile
       // Row sums at the reference m_ref: .x sums the probabilities (-> LSE); .y
       // normalises O and differs from .x by the bf16 rounding of each half's largest
       // probability: under the lagging reference a dominant key has P up to 2^8, and
@@ -664,7 +777,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ++seq;
           if (lane == 0) votes[x * 16 + (seq & 3) * 4 + wq] = (seq << 2) | vote;
           if (vote == 3) {
-            decision = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status);
+            decision = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status, kWaitLimitNs);
             if (decision < 0) { ok = false; break; }
             skip_all = decision == 3;
             if (!skip_all) pf_load_scores<CAUSAL>(taddr_s, s, key0, off + row, off + row0, n_keys);
@@ -682,6 +795,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[L::bPFull + x]);
             if (p.skip_mask && t == 0) pf_write_skip_mask<CAUSAL>(p, b, hq, qb * 2 + x, j, last_row, 3);
+            if (t == 0) n_skipped += pf_count_skipped<CAUSAL>(p, j, last_row, 3);
             continue;
           }
         }
@@ -763,13 +877,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if constexpr (SKIP) {
           // The other warps voted before their exponentials, so by now the
           // decision is normally complete; fold in the sums of the kept halves.
-          const int d = decision >= 0 ? decision : pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status);
+          const int d = decision >= 0 ? decision
+                                      : pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status,
+                                                         kWaitLimitNs);
           if (d < 0) { ok = false; break; }
           l = sum2_add(l, sum2_kept(hsum, d));
           if (p.skip_mask && t == 0) pf_write_skip_mask<CAUSAL>(p, b, hq, qb * 2 + x, j, last_row, d);
+          if (t == 0) n_skipped += pf_count_skipped<CAUSAL>(p, j, last_row, d);
         }
       }
       if (!ok) break;
+
+      if (SKIP && t == 0 && n_skipped && p.skipped_tiles) atomicAdd(p.skipped_tiles, (unsigned long long)n_skipped);
 
       // ---------------------------------------------------------- epilogue
       if (!mbar_wait(&bars[L::bPVDone + x], pvd_ph, no_abort, p.status)) { ok = false; break; }

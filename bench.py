@@ -73,6 +73,22 @@ def load_profile_traffic():
     return {}
 
 
+def physical_gpu_id(local):
+    """The nvidia-smi --id of CUDA device ``local``: its UUID when torch reports one
+    (right under any CUDA_VISIBLE_DEVICES mapping), else the entry of
+    CUDA_VISIBLE_DEVICES, else the index itself."""
+    try:
+        uuid = str(torch.cuda.get_device_properties(local).uuid)
+        if uuid and uuid != "None":
+            return uuid if uuid.startswith(("GPU-", "MIG-")) else "GPU-" + uuid
+    except (AttributeError, RuntimeError, AssertionError):
+        pass
+    visible = [x.strip() for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    if local < len(visible):
+        return visible[local]
+    return str(local)
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle sampling during the timed region."""
 
@@ -80,16 +96,24 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
+    def __init__(self, index, fallback=None):
         self.index = index
+        self.fallback = fallback
         self.proc = None
         self.lines = []
 
+    def _spawn(self, gpu_id):
+        return subprocess.Popen(
+            ["nvidia-smi", f"--id={gpu_id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader", "-lms", "100"],
+            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.proc = self._spawn(self.index)
+            time.sleep(0.2)
+            if self.proc.poll() is not None and self.fallback is not None:   # id not accepted
+                self.index = self.fallback
+                self.proc = self._spawn(self.index)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except (OSError, FileNotFoundError):
@@ -122,7 +146,7 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "gpu": str(self.index)}
 
 
 def dist_setup(n_gpus):
@@ -257,7 +281,7 @@ def run_gpu(args, world, rank, local):
         decode_call()
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(physical_gpu_id(local), fallback=str(local))
     clocks.start()
     time.sleep(0.3)
     dist_barrier(world)

@@ -21,12 +21,14 @@
  * PART03). Hkv == Hq is MHA, Hkv == 1 is MQA.
  *
  * Optional BLASST tile skip ("高效部署稀疏注意力加速方案：BLASST方法详解与实践指南",
- * 架构与组件): with lambda > 0, a tile of 64 keys is skipped -- no P V product, and
- * no exponentials wherever the decision is known before they would be computed --
- * when exp(tile_rowmax - running_max) < lambda for every row of its decision unit.
- * (The V tile is still read in this version: it travels with K.) The running
- * maximum is over the unit's tiles already kept, in ascending key order.
- * lambda == 0 computes the dense result.
+ * 架构与组件): with lambda > 0, a tile of 64 keys is skipped -- its V rows are not
+ * loaded, and it costs no P V product and no exponentials -- when
+ * exp(tile_rowmax - running_max) < lambda for every row of its decision unit.
+ * The running maximum is over the unit's tiles already kept, in ascending key
+ * order. lambda == 0 computes the dense result. (Exceptions, stated at the entry
+ * points: a V tile shared by several decision units is loaded while one of them
+ * keeps it, and a prefill warp whose rows keep a tile computes its
+ * exponentials before the other warps' votes are in.)
  *
  * Common conventions
  *   - Every pointer is a DEVICE pointer owned by the caller. The library never
@@ -43,9 +45,12 @@
  *   - Return value: ATTN_OK, or an error code. Argument errors are detected on
  *     the host before anything is enqueued. Errors found on the device
  *     (out-of-range block-table entries, a pipeline wait that timed out) are
- *     reported through `device_status` when given, and always through the
- *     library's device status word (attn_read_device_status). No kernel traps.
- *     The status words keep the largest code recorded.
+ *     reported through `device_status` when given, and through the library's
+ *     device status word once attn_set_library_status(1) has switched it on.
+ *     No kernel traps. The status words keep the largest code recorded.
+ *   - By default the library keeps no state that calls share: its device status
+ *     word is written only when switched on, and the one fixed scratch array
+ *     belongs to attn_decode_paged_noalloc alone.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -98,14 +103,19 @@ int attn_prefill(const void* q, const void* k, const void* v, void* o, float* ls
  *   skip_mask  [B][Hq][ceil(S/128)][ceil(S/64)] uint8, may be NULL. For every
  *              visited tile the kernel writes 1 (skipped) or 0 (kept); entries
  *              of tiles never visited are left untouched.
+ *   skipped_tiles  one unsigned 64-bit counter on the device, may be NULL
+ *              (8-byte aligned): the number of skipped decisions is added to it
+ *              (the caller zeroes it).
  *   device_status  int on the device, may be NULL; set (never cleared) to a
  *              device-side error code.
  * The output and LSE are those of attention restricted to the kept keys.
+ * The two query tiles of one 256-row block of a head share every K/V tile
+ * load: a 64-key half of V is loaded when either of the two keeps it.
  */
 int attn_prefill_blasst(const void* q, const void* k, const void* v, void* o, float* lse,
                         int B, int Hq, int Hkv, int S, int D, int causal, float scale,
-                        float lambda, uint8_t* skip_mask, int* device_status,
-                        void* stream);
+                        float lambda, uint8_t* skip_mask, unsigned long long* skipped_tiles,
+                        int* device_status, void* stream);
 
 /*
  * attn_prefill_paged -- chunked (append) prefill over a paged KV cache
@@ -168,10 +178,25 @@ int attn_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_
  * reset by the library on every call) and those partials:
  *   fp32 [num_seqs][max_splits][Hq][D] (padded to 256 B) + fp32 [num_seqs][max_splits][Hq]
  * with max_splits = ceil(max_pages_per_seq * page_size / split_tokens).
- * Returns 0 for invalid arguments.
+ * Returns 0 for invalid arguments or a size that does not fit a size_t.
  */
 size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq,
                                    int page_size, int split_tokens);
+
+/*
+ * attn_decode_blasst_workspace_bytes -- scratch needed by attn_decode_paged and
+ * attn_decode_paged_blasst_heads on their tile-skip path (lambda > 0, a
+ * skip_mask or a skipped_tiles counter, or the per-head entry point). That path
+ * runs in two passes: the first computes the scaled scores of every cached
+ * token and query head, and the row maxima of every 64-token tile and of every
+ * work chunk; the second derives the decisions from the maxima and reads V only
+ * for kept tiles. The workspace holds the scores (fp32
+ * [num_seqs][Hq][padded tokens]), the maxima, and one partial (O, LSE) per
+ * (sequence, query head, chunk); a chunk is at most 256 tokens and divides
+ * split_tokens. Returns 0 for invalid arguments or an overflowing size.
+ */
+size_t attn_decode_blasst_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq,
+                                          int page_size, int split_tokens);
 
 /*
  * attn_decode_paged -- single-token decode over a paged KV cache (split-KV
@@ -193,15 +218,21 @@ size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_pe
  *                64-token tiles, the running maximum restarts at each split
  *   split_tokens multiple of 64 (>= 64): tokens per split
  *   o            [num_seqs][Hq][D] bf16, lse [num_seqs][Hq] fp32 (lse may be NULL)
- *   workspace    device scratch of at least attn_decode_workspace_bytes(...)
- *                bytes, 16-byte aligned; contents on entry are ignored
+ *   workspace    device scratch, 16-byte aligned, contents on entry ignored, of at
+ *                least attn_decode_workspace_bytes(...) bytes on the dense path and
+ *                attn_decode_blasst_workspace_bytes(...) bytes on the skip path
  *   skip_mask    [num_seqs][Hkv][ceil(max_pages_per_seq*page_size/64)] uint8,
  *                may be NULL: 1 skipped / 0 kept for every visited tile; other
  *                entries untouched
+ *   skipped_tiles  device counter, may be NULL (see attn_prefill_blasst)
  *   device_status  may be NULL (see attn_prefill_blasst)
  * A block_table entry outside [0, num_pages) is never dereferenced: its
  * tokens are treated as absent and ATTN_ERR_DEVICE_BOUNDS is raised.
- * Hq / Hkv must be 1, 2, 4, 8 or 16.
+ * Hq / Hkv must be 1, 2, 4, 8 or 16. On the skip path with Hq / Hkv <= 8 a
+ * skipped tile's V rows are not read; with Hq / Hkv = 16 the skip path runs a
+ * one-pass kernel that still reads them.
+ * Pointers: q, pages, o and workspace 16-byte aligned; block_table, seq_lens
+ * and lse 4-byte aligned; skipped_tiles 8-byte aligned.
  */
 int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                       const int32_t* block_table, const int32_t* seq_lens,
@@ -209,7 +240,8 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                       int max_pages_per_seq, int num_pages, float scale, float lambda,
                       int split_tokens, void* o, float* lse,
                       void* workspace, size_t workspace_bytes,
-                      uint8_t* skip_mask, int* device_status, void* stream);
+                      uint8_t* skip_mask, unsigned long long* skipped_tiles,
+                      int* device_status, void* stream);
 
 /*
  * attn_decode_paged_blasst_heads -- attn_decode_paged with the BLASST tile skip
@@ -218,11 +250,13 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
  * instead of the G heads that share a KV head. The page states the rule for
  * the rows of a tile without fixing which rows share a tile in decode; this is
  * the narrowest reading. A head that drops a 64-token tile gets no probability
- * mass from it; the tile's K and V are still read while another head of the
- * group keeps it.
- * Arguments as attn_decode_paged, except:
+ * mass from it; the tile's V rows are still read while another head of the
+ * same KV head keeps it, and not read once all of them drop it.
+ * Arguments as attn_decode_paged (the workspace is always the skip path's),
+ * except:
  *   skip_mask    [num_seqs][Hq][ceil(max_pages_per_seq*page_size/64)] uint8, may be
  *                NULL: 1 skipped / 0 kept for every visited (head, tile)
+ *   skipped_tiles  counts skipped (query head, tile) decisions
  *   lambda       in [0, 1); 0 decides nothing away (the dense result)
  */
 int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const void* v_pages,
@@ -231,7 +265,8 @@ int attn_decode_paged_blasst_heads(const void* q, const void* k_pages, const voi
                                    int max_pages_per_seq, int num_pages, float scale, float lambda,
                                    int split_tokens, void* o, float* lse,
                                    void* workspace, size_t workspace_bytes,
-                                   uint8_t* skip_mask, int* device_status, void* stream);
+                                   uint8_t* skip_mask, unsigned long long* skipped_tiles,
+                                   int* device_status, void* stream);
 
 /*
  * attn_decode_paged_fp8 -- attn_decode_paged (dense) over a cache stored as
@@ -273,9 +308,10 @@ int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_code
  * holds until the process exits.
  *
  * Arguments, layouts, results and errors are those of attn_decode_paged,
- * minus workspace / workspace_bytes. A call whose
+ * minus workspace / workspace_bytes and skipped_tiles. A call whose
  * attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages_per_seq, page_size,
- * split_tokens) exceeds ATTN_NOALLOC_SCRATCH_BYTES returns
+ * split_tokens) -- attn_decode_blasst_workspace_bytes(...) with lambda > 0 or a
+ * skip_mask -- exceeds ATTN_NOALLOC_SCRATCH_BYTES returns
  * ATTN_ERR_INVALID_ARG before anything is enqueued (use a larger split_tokens
  * or attn_decode_paged).
  *
@@ -296,12 +332,38 @@ int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_
                               uint8_t* skip_mask, int* device_status, void* stream);
 
 /*
+ * attn_set_library_status -- switch the library's device status word on the
+ * current device on (enable != 0) or off (the default). While it is on, every
+ * kernel of the library also records its device-side errors there (the largest
+ * code wins), so independent callers on one device see each other's errors;
+ * the per-call device_status arguments need no switch. Synchronous (a small
+ * host-to-device copy).
+ */
+int attn_set_library_status(int enable);
+
+/*
  * attn_read_device_status -- read (and, if clear != 0, reset to ATTN_OK) the
  * library's device status word on the current device. Synchronises the
- * device. Every kernel of the library records device-side errors in it (the
- * largest code wins).
+ * device.
  */
 int attn_read_device_status(int* status_out, int clear);
+
+/*
+ * attn_debug_prefill_timeout -- TEST ONLY: attn_prefill (dense) with a shorter
+ * pipeline wait limit and, when withhold_step >= 0, one K/V ring step of every
+ * CTA left out by the producer: its copy is never issued and its barrier never
+ * armed, so the MMA issuer's wait for it runs out. No production caller needs
+ * it. It exercises the kernels' abort path without faulting or hanging the GPU:
+ * each wait gives up after wait_limit_ns (1 us .. 2 s), the CTA records
+ * ATTN_ERR_TIMEOUT in device_status, lets its copies in flight land, waits for
+ * its tensor-core work to finish, releases its tensor memory and returns. The
+ * output is then undefined; later calls on the same context are unaffected.
+ * Arguments otherwise as attn_prefill.
+ */
+int attn_debug_prefill_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int Hq, int Hkv, int S, int D, int causal, float scale,
+                               unsigned long long wait_limit_ns, int withhold_step,
+                               int* device_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -8,7 +8,7 @@ error, then refined by a few Lawson (iteratively reweighted) steps towards the
 minimax solution. The probabilities it produces are rounded to bf16 (relative
 step 2^-8), so a relative error near 1e-4 is far below what is kept.
 
-Run: python fit_exp2_poly.py  -> prints the coefficients c0..c3 and the max
+Run: python tests/exp2_poly_fit.py  -> prints the coefficients c0..c3 and the max
 relative error over [-1/2, 1/2].
 """
 

@@ -45,7 +45,7 @@ def test_status_strings(lib):
     for code, name in binding.STATUS.items():
         assert lib.attn_status_string(code).decode() == name
     assert lib.attn_status_string(99).decode() == "ATTN_ERR_UNKNOWN"
-    assert lib.attn_abi_version() == 1
+    assert lib.attn_abi_version() == 2
 
 
 def _prefill(lib, **kw):
@@ -69,8 +69,14 @@ def test_prefill_rejects_unsupported_head_dim(lib):
 def test_prefill_blasst_rejects_bad_lambda(lib):
     for lam in (-0.1, 1.0, 2.0, float("nan")):
         st = lib.attn_prefill_blasst(FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, 64, 1, 0.125, lam, None, None,
-                                     None)
+                                     None, None)
         assert st == INVALID
+
+
+def test_prefill_blasst_rejects_a_misaligned_counter(lib):
+    st = lib.attn_prefill_blasst(FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, 64, 1, 0.125, 0.1, None,
+                                 ctypes.c_void_p((1 << 20) + 4), None, None)
+    assert st == INVALID
 
 
 def test_workspace_bytes(lib):
@@ -85,6 +91,36 @@ def test_workspace_bytes(lib):
     for bad in [(0, hq, d, mp, ps, sp), (n, hq, 96, mp, ps, sp), (n, hq, d, mp, 24, sp), (n, hq, d, mp, ps, 100),
                 (n, hq, d, 0, ps, sp)]:
         assert lib.attn_decode_workspace_bytes(*bad) == 0
+        assert lib.attn_decode_blasst_workspace_bytes(*bad) == 0
+
+
+def test_workspace_bytes_overflow_returns_zero(lib):
+    # 2^31 sequences x 2^31 heads x ... does not fit a size_t: 0, never a wrapped small size
+    big = 2 ** 31 - 1
+    assert lib.attn_decode_workspace_bytes(big, big, 128, 2 ** 20, 256, 64) == 0
+    assert lib.attn_decode_blasst_workspace_bytes(big, big, 128, 2 ** 20, 256, 64) == 0
+
+
+def _blasst_layout(n, hq, d, mp, ps, sp):
+    """The tile-skip workspace as the header documents it (chunk choice included)."""
+    cap = mp * ps
+    c = next((x for x in (256, 192, 128) if sp % x == 0), 64)
+    while c % 128 == 0 and n * hq * -(-cap // c) < 8192:
+        c //= 2
+    chunks, tiles = -(-cap // c), -(-cap // 64)
+    r256 = lambda x: -(-x // 256) * 256
+    parts = [n * hq * chunks * d * 4, n * hq * chunks * 4, n * hq * tiles * 64 * 4, n * hq * tiles * 4,
+             n * hq * chunks * 4]
+    return 256 + sum(r256(x) for x in parts), c
+
+
+@pytest.mark.parametrize("args", [(64, 32, 128, 512, 16, 256), (1, 32, 128, 2048, 16, 2048),
+                                  (8, 16, 64, 40, 64, 320), (3, 8, 128, 10, 16, 64)])
+def test_blasst_workspace_bytes(lib, args):
+    want, _ = _blasst_layout(*args)
+    dense = lib.attn_decode_workspace_bytes(*args)
+    assert lib.attn_decode_blasst_workspace_bytes(*args) == max(want, dense)
+    assert ab.binding.decode_blasst_workspace_bytes(*args) == max(want, dense)
 
 
 def _decode(lib, **kw):
@@ -93,15 +129,26 @@ def _decode(lib, **kw):
     a.update(kw)
     return lib.attn_decode_paged(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["N"], a["Hq"], a["Hkv"], a["D"],
                                  a["ps"], a["mp"], a["P"], a["scale"], a["lam"], a["split"], a["o"], a["lse"],
-                                 a["ws"], a["wsb"], None, None, None)
+                                 a["ws"], a["wsb"], None, a.get("cnt"), None, None)
 
 
 @pytest.mark.parametrize("bad", [dict(q=None), dict(bt=None), dict(sl=None), dict(ws=None), dict(N=0),
                                  dict(Hq=6, Hkv=4), dict(ps=24), dict(ps=0), dict(split=96), dict(split=0),
                                  dict(mp=0), dict(P=0), dict(lam=1.0), dict(lam=-0.5), dict(wsb=16),
-                                 dict(kp=ctypes.c_void_p((1 << 20) + 4))])
+                                 dict(kp=ctypes.c_void_p((1 << 20) + 4)), dict(bt=ctypes.c_void_p((1 << 20) + 2)),
+                                 dict(sl=ctypes.c_void_p((1 << 20) + 1)), dict(lse=ctypes.c_void_p((1 << 20) + 2)),
+                                 dict(cnt=ctypes.c_void_p((1 << 20) + 4)), dict(N=2 ** 20, Hq=2 ** 12, Hkv=2 ** 10)])
 def test_decode_rejects_bad_arguments(lib, bad):
     assert _decode(lib, **bad) == INVALID
+
+
+def test_decode_skip_path_needs_the_larger_workspace(lib):
+    args = (4, 8, 128, 8, 16, 64)
+    dense = lib.attn_decode_workspace_bytes(*args)
+    skip = lib.attn_decode_blasst_workspace_bytes(*args)
+    assert skip > dense > 0
+    assert _decode(lib, lam=0.2, wsb=dense) == INVALID
+    assert _decode(lib, cnt=FAKE, wsb=dense) == INVALID       # a counter selects the skip path too
 
 
 @pytest.mark.parametrize("bad", [dict(D=80), dict(Hq=24, Hkv=1), dict(Hq=6, Hkv=2)])
@@ -115,6 +162,22 @@ def test_valid_arguments_without_a_device_report_cuda_error(lib):
         pytest.skip("a device is present")
     assert _prefill(lib) == CUDA
     assert _decode(lib) == CUDA
+    assert _decode(lib, lam=0.3) == CUDA
+    assert lib.attn_set_library_status(1) == CUDA
+
+
+@pytest.mark.parametrize("limit", [0, 999, 2_000_000_001])
+def test_debug_timeout_rejects_limits_out_of_range(lib, limit):
+    st = lib.attn_debug_prefill_timeout(FAKE, FAKE, FAKE, FAKE, None, 1, 2, 1, 128, 128, 1, 0.088, limit, 1,
+                                        None, None)
+    assert st == INVALID
+
+
+def test_noalloc_rejects_a_skip_call_beyond_its_scratch(lib):
+    # the skip path also keeps the scores: 64 x 32 x 8192 x 4 B alone is 64 MiB
+    st = lib.attn_decode_paged_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 32, 8, 128, 16, 512, 1024, 0.088, 0.3,
+                                       2048, FAKE, None, None, None, None)
+    assert st == INVALID
 
 
 def test_binding_fails_loudly_when_library_missing(monkeypatch):

@@ -8,7 +8,7 @@ import os
 
 import numpy as np
 
-from attention_online_softmax_fwd_b200.csrc import fit_exp2_poly
+import exp2_poly_fit as fit_exp2_poly
 
 CSRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                     "attention_online_softmax_fwd_b200", "csrc", "common.cuh")

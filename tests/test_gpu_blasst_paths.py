@@ -1,0 +1,111 @@
+"""Tile-skip paths on the GPU against the float64 oracle: the two-pass decode
+over every head layout it serves (and the one-pass kernel kept for 16 query
+heads per KV head), the skipped-decision counters, and the library's status
+word being opt-in."""
+
+import numpy as np
+import pytest
+import torch
+
+import attention_online_softmax_fwd_b200 as ab
+from attention_online_softmax_fwd_b200 import inputs as gen
+from oracle import attn_oracle as orc
+from parity_util import compare_blasst
+
+pytestmark = pytest.mark.gpu
+
+LENS = [1, 63, 64, 65, 700, 2049, 0, 1300]
+
+
+def _cache(Hq, Hkv, D, ps, seed):
+    """Ragged sequences (one empty) of N(0, 1) K/V; the queries are scaled by 3 so
+    that scores spread and later tiles fall below their split's running maximum."""
+    c = gen.paged_decode_inputs(len(LENS), Hq, Hkv, D, ps, 0, 0, seed=seed, lens=LENS)
+    c.q = (c.q.float() * 3.0).to(torch.bfloat16)
+    return c
+
+
+def _run(c, dev, lam, split, rows):
+    args = [t.to(dev) for t in (c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens)]
+    counter = torch.zeros(1, dtype=torch.int64, device=dev)
+    scale = gen.attn_scale(c.q.shape[-1])
+    o, lse, mask = ab.decode_paged_blasst(*args, lam, scale=scale, split_tokens=split, rows_per_unit=rows,
+                                          skipped_tiles=counter)
+    torch.cuda.synchronize()
+    return o, lse, mask, int(counter.item()), scale
+
+
+# (Hq, Hkv, D, page size): groups of 4 KV heads (Hkv % 4 == 0), single KV heads
+# (Hkv = 2, 12 / 4 = 3 groups), G = 1, 2, 4, 8 on the two-pass kernels; G = 16 on
+# the one-pass kernel
+SHAPES = [(8, 2, 128, 16), (32, 8, 64, 64), (8, 8, 128, 256), (64, 8, 128, 16), (24, 12, 128, 64),
+          (16, 8, 64, 16), (16, 1, 128, 16)]
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,ps", SHAPES)
+@pytest.mark.parametrize("split", [64, 320, 2048])
+@pytest.mark.parametrize("rows", ["group", "head"])
+def test_decode_blasst_layouts(cuda_device, Hq, Hkv, D, ps, split, rows):
+    c = _cache(Hq, Hkv, D, ps, seed=5000 + Hq + D + ps)
+    o, lse, mask, counted, scale = _run(c, cuda_device, 0.5, split, rows)
+    o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens,
+                                                            ps, scale, 0.5, split, rows_per_unit=rows)
+    o_ref[6], lse_ref[6] = 0.0, -np.inf        # the empty sequence
+
+    def with_mask(m):
+        of, lf = orc.decode_paged_with_skip_mask(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens, ps, scale,
+                                                 m, rows_per_unit=rows)
+        of[6], lf[6] = 0.0, -np.inf
+        return of, lf
+
+    st = compare_blasst(o, lse, mask, o_ref, lse_ref, m_ref, margin, with_mask,
+                        label=f"Hq={Hq} Hkv={Hkv} D={D} ps={ps} split={split} {rows}")
+    assert counted == st["skipped_gpu"], "the counter adds one per skipped decision"
+    if split > 64:
+        assert st["skipped"] > 0
+
+
+def test_decode_blasst_lambda_zero_keeps_everything(cuda_device):
+    c = _cache(32, 8, 128, 16, seed=5100)
+    o, lse, mask, counted, scale = _run(c, cuda_device, 0.0, 320, "group")
+    o_ref, lse_ref = orc.decode_paged(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens, 16, scale)
+    o_ref[6], lse_ref[6] = 0.0, -np.inf
+    assert counted == 0 and not (mask == 1).any()
+    from parity_util import compare_output
+    compare_output(o, o_ref, lse, lse_ref, label="lambda 0, two passes")
+
+
+def test_decode_blasst_repeatable(cuda_device):
+    c = _cache(32, 8, 128, 16, seed=5200)
+    a = _run(c, cuda_device, 0.5, 2048, "group")
+    b = _run(c, cuda_device, 0.5, 2048, "group")
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2]) and a[3] == b[3]
+
+
+def test_prefill_skipped_counter(cuda_device):
+    q, k, v = gen.peaked_prefill_inputs(1, 4, 2, 1100, 128, seed=3200, amp=8.0, period=1 << 30)
+    dev = cuda_device
+    counter = torch.zeros(1, dtype=torch.int64, device=dev)
+    o, lse, mask = ab.prefill_blasst(q.to(dev), k.to(dev), v.to(dev), 0.3, causal=True,
+                                     scale=gen.attn_scale(128), skipped_tiles=counter)
+    torch.cuda.synchronize()
+    assert int(counter.item()) == int((mask == 1).sum().item()) > 0
+
+
+def test_library_status_word_is_opt_in(cuda_device):
+    c = gen.paged_decode_inputs(4, 8, 2, 128, 16, 100, 300, seed=5300)
+    c.block_table[1, 2] = c.num_pages + 5      # out of range: never dereferenced, reported
+    args = [t.to(cuda_device) for t in (c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens)]
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ab.binding.set_library_status(False)
+    ab.binding.read_device_status(clear=True)
+    ab.decode_paged(*args, split_tokens=64, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 4                               # the caller's own word
+    assert ab.binding.read_device_status(clear=True) == 0        # the library's stays untouched
+    ab.binding.set_library_status(True)
+    try:
+        ab.decode_paged(*args, split_tokens=64)
+        assert ab.binding.read_device_status(clear=True) == 4
+    finally:
+        ab.binding.set_library_status(False)

@@ -134,11 +134,13 @@ def test_decode_bad_page_raises_device_status(cuda_device):
     cache.block_table[2, 0] = -7
     q, kp, vp, bt, sl = _to(cache, cuda_device)
     status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ab.binding.set_library_status(True)
     ab.binding.read_device_status(clear=True)
     o, lse = ab.decode_paged(q, kp, vp, bt, sl, split_tokens=64, device_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 4                        # ATTN_ERR_DEVICE_BOUNDS
     assert ab.binding.read_device_status(clear=True) == 4
+    ab.binding.set_library_status(False)
     # sequences with valid tables are unaffected
     o_ref, lse_ref = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens,
                                       16, gen.attn_scale(128), seqs=[0, 3])

@@ -108,10 +108,12 @@ def test_decode_fp8_bad_page_raises_device_status(cuda_device):
     cache.block_table[2, 0] = -7
     kc, ks, vc, vs = _quantized(cache)
     status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ab.binding.set_library_status(True)
     ab.binding.read_device_status(clear=True)
     o, lse, scale = _run(cache, kc, ks, vc, vs, cuda_device, 64, status=status)
     assert int(status.item()) == 4                        # ATTN_ERR_DEVICE_BOUNDS
     assert ab.binding.read_device_status(clear=True) == 4
+    ab.binding.set_library_status(False)
     o_ref, lse_ref = orc.decode_paged_fp8(cache.q, kc, vc, ks, vs, cache.block_table, cache.seq_lens, 16, scale,
                                           seqs=[0, 3])
     compare_output(o[[0, 3]], o_ref[[0, 3]], lse[[0, 3]], lse_ref[[0, 3]])
