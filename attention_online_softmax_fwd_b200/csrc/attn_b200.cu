@@ -301,20 +301,25 @@ bool blasst_layout(int num_seqs, int Hq, int D, int max_pages, int page_size, in
 // as a programmatic dependent of the split kernel: it is scheduled while the split
 // kernel's last CTAs run and waits (griddepcontrol.wait) for that grid to finish
 // and its writes to be visible before it reads the partials.
+// Sixteen warps per (sequence, head) when a row has more than 64 partials (long
+// sequences at small splits), four otherwise.
 template <int D>
 int launch_merge(const DecodeParams& p, cudaStream_t stream) {
   const long long pairs = (long long)p.num_seqs * p.Hq;
+  const bool wide = p.max_splits > 64;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(pairs));
-  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.blockDim = dim3((wide ? 16 : 4) * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, decode_merge_kernel<D>, p) != cudaSuccess) return ATTN_ERR_CUDA;
+  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 16>, p)
+                             : cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 4>, p);
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
   return launch_status();
 }
 

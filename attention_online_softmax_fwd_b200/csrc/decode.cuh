@@ -589,13 +589,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // Combine the split partials of one (sequence, query head) per CTA: each
 // partial is a normalised O row (fp32) with its log2-sum-exp; the result is
 // sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M), M the largest lse_s. Warp w
-// takes splits w, w + 4, ... in chunks of kMergeChunk, loading each chunk's
+// takes splits w, w + W, ... in chunks of kMergeChunk, loading each chunk's
 // lse values and O rows together (one memory round trip per chunk), and keeps a
-// running maximum; the four warps then combine in a fixed order (deterministic).
-constexpr int kMergeWarps = 4;
+// running maximum; the W warps then combine in a fixed order (deterministic).
+// W = 4 serves batches of many sequences; W = 16 puts four times as many
+// partials in flight for the few rows of a long single sequence.
 constexpr int kMergeChunk = 8;   // splits per warp in flight
-template <int D>
-__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const DecodeParams p) {
+template <int D, int W = 4>
+__global__ void __launch_bounds__(W * 32) decode_merge_kernel(const DecodeParams p) {
+  constexpr int kMergeWarps = W;
   constexpr int DL = D / 32;   // floats per lane: 4 (D = 128) or 2 (D = 64)
   __shared__ float sh_m[kMergeWarps], sh_w[kMergeWarps];
   __shared__ __align__(16) float sh_acc[kMergeWarps][D];

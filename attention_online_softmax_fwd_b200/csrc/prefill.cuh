@@ -185,6 +185,10 @@ __device__ __forceinline__ int pf_dropped_by_both(const volatile int* votes, int
       d &= w.x & w.y & w.z & w.w;
     }
     if (in) return d & 3;
+    // the votes come once the softmax warps have the tile's row maxima, often a few hundred
+    // cycles away: sleep between polls, so that this warp takes no issue slots from the
+    // softmax warps that share its SM sub-partition
+    __nanosleep(64);
     if (i == 0) {
       t0 = global_timer_ns();
     } else if ((i & 31u) == 0) {
@@ -200,8 +204,10 @@ __device__ __forceinline__ int pf_dropped_by_both(const volatile int* votes, int
 
 // The order of one item's K and V tiles in the ring: K_0 .. K_{L-1}, then V_j and
 // K_{j+L} in turn, then the last V tiles. With L = 2 each K_{j+1} is loaded just
-// before V_j; the tile skip uses L = 3, so that the skip decision on tile j is in
-// before V_j is due and a dropped tile's V need not be loaded.
+// before V_j. (A larger L would let every skip decision arrive before its V is
+// due, but with three ring slots it leaves V_j waiting for the slot of K_{j+1}
+// and exposes the V latency on every tile: 1.5x the dense time when nothing is
+// skipped.)
 template <int L>
 __device__ __forceinline__ void pf_ring_step(int step, int n, bool& is_k, int& tile) {
   const int a = n < L ? n : L;
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   using L = PrefillSmem<D>;
   constexpr int NS = L::kStages;
   constexpr int kTmemCols = 512;
-  constexpr int kLead = SKIP ? 3 : 2;   // K tiles loaded before the first V (pf_ring_step)
+  constexpr int kLead = 2;   // K tiles loaded before the first V (pf_ring_step)
 
 
   extern __shared__ uint8_t smem_raw[];
@@ -514,6 +520,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         uint32_t qe_bits = 3u;
         uint32_t pend_mask = 0, pend_ph = 0;
         int vseq[2] = {0, 0};   // SKIP: the tiles each softmax warpgroup has voted on (its vote sequence)
+        bool prev_dropped = false;          // SKIP: both query tiles dropped the whole previous V tile
+        int pend_tag0 = 0, pend_tag1 = 0;   // SKIP: votes of a V tile loaded without its decision
         int gstep = 0;          // ring steps of this CTA (for the test-only withheld step)
         bool ok = true;
         for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
@@ -547,13 +555,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             int halves = 3;   // bit h: 64-key half h of the tile is loaded
             if constexpr (SKIP) {
               if (!is_k) {
-                // V_tile is loaded only for the halves that one of the two query tiles keeps; both
-                // softmax warpgroups have voted on the tile by now (K runs kLead tiles ahead)
+                // V_tile is due before the softmax warps have voted on it. After a tile that both
+                // query tiles dropped, the producer waits for the votes and loads only the halves
+                // that one of the two keeps, so a run of dropped tiles reads no V; after a kept
+                // tile it loads the whole tile at once, which keeps the dense pipeline.
                 const int tag0 = tile < nkv0 ? ++vseq[0] : 0;   // 0: this query tile does not visit it
                 const int tag1 = tile < nkv1 ? ++vseq[1] : 0;
-                const int dropped = pf_dropped_by_both(votes, tag0, tag1, abort_flag, p.status, p.wait_ns);
-                if (dropped < 0) { ok = false; break; }
-                halves = ~dropped & 3;
+                if (tile == 0) {
+                  prev_dropped = false;   // a unit's first tile is never dropped
+                } else if (pend_tag0 | pend_tag1) {
+                  // the previous tile's votes (loaded at once): in by now, since Q K^T of this tile,
+                  // issued after they were cast, has completed
+                  const int d = pf_dropped_by_both(votes, pend_tag0, pend_tag1, abort_flag, p.status, p.wait_ns);
+                  if (d < 0) { ok = false; break; }
+                  prev_dropped = d == 3;
+                }
+                pend_tag0 = pend_tag1 = 0;
+                if (prev_dropped) {
+                  const int dropped = pf_dropped_by_both(votes, tag0, tag1, abort_flag, p.status, p.wait_ns);
+                  if (dropped < 0) { ok = false; break; }
+                  halves = ~dropped & 3;
+                  prev_dropped = dropped == 3;
+                } else {
+                  pend_tag0 = tag0;   // loaded without waiting; its votes are read at the next V
+                  pend_tag1 = tag1;
+                }
               }
             }
             if (!mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status, p.wait_ns)) {

@@ -391,8 +391,9 @@ def run_gpu(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_extras:
         line["decode_fp8"] = fp8_decode_report(dev, peaks, cache, flush)
         line["chunked_prefill_paged"] = chunked_prefill_report(dev, peaks)
+        line["mha_prefill"] = mha_prefill_report(dev, peaks)
     if rank == 0 and world == 1 and not args.no_blasst:
-        line["blasst_long_context"] = blasst_long_context_report(dev)
+        line["blasst_long_context"] = blasst_long_context_report(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfs, gbs, secs, desc = oracle_sample(int(args.cpu_heads), 4)
         line["cpu_baseline"] = {"value": tfs, "unit": "TFLOP/s", "cores": cpu_threads()[0], "kind": "oracle",
@@ -473,87 +474,122 @@ def chunked_prefill_report(dev, peaks, reps=5):
             "ms": ms, "tflops": tf, "flops": fl, "frac_of_measured_bf16": tf / peaks["bf16_tflops"]}
 
 
-def blasst_long_context_report(dev, reps=3):
-    """Long-context BLASST workload (B=1, Hq=32, Hkv=8, S=32768, D=128, 64-key tiles):
-    prefill and the decode of the last row at lambda in {0, 0.1, 0.3}. Reports the
-    time, the skipped fraction of visited tiles and the error against lambda = 0."""
+def mha_prefill_report(dev, peaks, reps=20):
+    """The MHA causal prefill shaped like a 7B Llama-2 layer (B=4, Hq=Hkv=32,
+    S=2048, D=128): 137.4 GFLOP per launch, L2 flushed before each launch."""
+    import attention_online_softmax_fwd_b200 as ab
+    c = gen.CONFIGS["mha_prefill_llama2_7b"]
+    B, Hq, Hkv, S, D = c["B"], c["Hq"], c["Hkv"], c["S"], c["D"]
+    q, k, v = [t.to(dev) for t in gen.prefill_inputs(B, Hq, Hkv, S, D, c["seed"])]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+    scale = gen.attn_scale(D)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ms = _timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale, out=o, lse=lse), dev, reps, flush)[0]
+    fl = prefill_flops(B, Hq, S, D)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": "mha_prefill_llama2_7b B4 Hq32 Hkv32 S2048 D128 causal", "kernel": "prefill_kernel<128,causal>",
+            "ms": ms, "tflops": tf, "flops_per_launch": fl, "frac_of_measured_bf16": tf / peaks["bf16_tflops"],
+            "frac_of_spec_2250": tf / SPEC_PEAKS["bf16_tflops"], "l2": "flushed before every launch"}
+
+
+def _timed(fn, dev, reps, flush=None):
+    """Median CUDA-event time (ms) of ``fn`` on the current stream, after one warm-up call."""
+    stream = torch.cuda.current_stream(dev)
+    out = fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        out = fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts), out
+
+
+def _decode_kept_bytes(mask, seq_lens, G, D, rows_per_unit, page_size, max_pages):
+    """Algorithmic bytes of a tile-skip decode: every cached K row, and the V rows
+    of the 64-token tiles that some query head of their KV head keeps."""
+    m = mask.cpu()
+    if rows_per_unit == "head":
+        n, hq, t = m.shape
+        m = m.view(n, hq // G, G, t)
+        kept = ((m == 0).any(dim=2))                     # a KV head's tile is loaded if one of its heads keeps it
+    else:
+        kept = (m == 0)
+    toks = 0
+    L = [int(x) for x in seq_lens]
+    for b, Lb in enumerate(L):
+        for t in range(-(-Lb // 64)):
+            n_tok = min(64, Lb - 64 * t)
+            toks += n_tok * int(kept[b, :, t].sum())
+    return sum(L) * kept.shape[1] * D * 2, toks * D * 2    # (K bytes, kept V bytes)
+
+
+def blasst_long_context_report(dev, peaks, reps=5):
+    """Long-context BLASST workload (B=1, Hq=32, Hkv=8, S=32768, D=128, 64-key tiles,
+    lambda in {0, 0.1, 0.3}): prefill, and the decode of the last row over the paged
+    cache at split_tokens = 2048 (the decision split of the workload; 256 as an
+    extra line), for the recipe input (4u on every 64th key) and a single dominant
+    key (12u on key 0). Reports times, skipped fractions, the kept-tile bytes the
+    decode reads, the error against lambda = 0 and the speedup over the dense path
+    (the dense decode at its fastest split, 256)."""
     import attention_online_softmax_fwd_b200 as ab
     c = gen.CONFIGS["blasst_long_context"]
     B, Hq, Hkv, S, D = c["B"], c["Hq"], c["Hkv"], c["S"], c["D"]
-    q_h, k_h, v_h = gen.peaked_prefill_inputs(B, Hq, Hkv, S, D, c["seed"], amp=4.0, period=64)
-    cache = gen.paged_from_contiguous(q_h[:, S - 1], k_h, v_h, page_size=c["page_size"], seed=c["seed"] + 1,
-                                      poison=False)
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    dargs = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    G = Hq // Hkv
     scale = gen.attn_scale(D)
-    split = 256   # 128 splits of the one sequence: enough work items for every SM
-    stream = torch.cuda.current_stream(dev)
-
-    def timed(fn):
-        fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            out = fn()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        return statistics.median(ts), out
-
     fl = prefill_flops(B, Hq, S, D)
-    dbytes = decode_bytes([S], Hq, Hkv, D, cache.max_pages)
-    report = {"workload": "blasst_long_context B1 Hq32 Hkv8 S32768 D128, tiles of 64 keys, decode split 256",
-              "prefill": {}, "decode": {}}
-    ms0, (o0, l0) = timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale))
-    dms0, (do0, dl0) = timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=split))
-    report["prefill"]["0.0"] = {"ms": ms0, "tflops": fl / (ms0 * 1e-3) / 1e12, "skipped_frac": 0.0}
-    report["decode"]["0.0"] = {"ms": dms0, "gbs": dbytes / (dms0 * 1e-3) / 1e9, "skipped_frac": 0.0}
-    for lam in (0.1, 0.3):
-        ms, (o, l, mask) = timed(lambda: ab.prefill_blasst(q, k, v, lam, causal=True, scale=scale))
-        vis = (mask != 2)
-        err = (o.float() - o0.float()).abs()
-        report["prefill"][str(lam)] = {
-            "ms": ms, "tflops_dense_equiv": fl / (ms * 1e-3) / 1e12,
-            "skipped_frac": float(((mask == 1) & vis).sum().item() / vis.sum().item()),
-            "max_abs_err_vs_dense": float(err.max().item()), "mean_abs_err_vs_dense": float(err.mean().item()),
-            "speedup_vs_dense": ms0 / ms}
-        dms, (do, dl, dmask) = timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split))
-        dvis = (dmask != 2)
-        derr = (do.float() - do0.float()).abs()
-        report["decode"][str(lam)] = {
-            "ms": dms, "gbs_dense_equiv": dbytes / (dms * 1e-3) / 1e9,
-            "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
-            "max_abs_err_vs_dense": float(derr.max().item()), "speedup_vs_dense": dms0 / dms}
-        hms, (ho, hl, hmask) = timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split,
-                                                                    rows_per_unit="head"))
-        hvis = (hmask != 2)
-        report["decode"][str(lam) + "_per_head"] = {
-            "ms": hms, "skipped_frac": float(((hmask == 1) & hvis).sum().item() / hvis.sum().item()),
-            "max_abs_err_vs_dense": float((ho.float() - do0.float()).abs().max().item()),
-            "speedup_vs_dense": dms0 / hms}
-
-    # The recipe above puts a raised key in every 64-key tile, so no tile can be
-    # dropped. A second input with a single dominant key at position 0 (12 u on
-    # key 0 and on all queries) shows the skip path when most tiles fall below
-    # the running maximum.
-    q_h, k_h, v_h = gen.peaked_prefill_inputs(B, Hq, Hkv, S, D, c["seed"] + 7, amp=12.0, period=S)
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    del q_h, k_h, v_h
-    sink = {"input": "12 u on key 0 and on all queries, no other raised keys", "prefill": {}}
-    ms0, (o0, l0) = timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale))
-    sink["prefill"]["0.0"] = {"ms": ms0, "tflops": fl / (ms0 * 1e-3) / 1e12}
-    for lam in (0.1, 0.3):
-        ms, (o, l, mask) = timed(lambda: ab.prefill_blasst(q, k, v, lam, causal=True, scale=scale))
-        vis = (mask != 2)
-        err = (o.float() - o0.float()).abs()
-        sink["prefill"][str(lam)] = {
-            "ms": ms, "tflops_dense_equiv": fl / (ms * 1e-3) / 1e12,
-            "skipped_frac": float(((mask == 1) & vis).sum().item() / vis.sum().item()),
-            "max_abs_err_vs_dense": float(err.max().item()), "mean_abs_err_vs_dense": float(err.mean().item()),
-            "speedup_vs_dense": ms0 / ms}
-    report["dominant_key_input"] = sink
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    report = {"workload": "blasst_long_context B1 Hq32 Hkv8 S32768 D128, tiles of 64 keys",
+              "decode_note": "decode bytes = every K row + V rows of kept (KV head, tile) pairs; L2 flushed",
+              "prefill_note": "prefill speedup against the dense kernel on the same input"}
+    for name, amp, period, seed in (("recipe", 4.0, 64, c["seed"]), ("dominant_key", 12.0, S, c["seed"] + 7)):
+        q_h, k_h, v_h = gen.peaked_prefill_inputs(B, Hq, Hkv, S, D, seed, amp=amp, period=period)
+        cache = gen.paged_from_contiguous(q_h[:, S - 1], k_h, v_h, page_size=c["page_size"], seed=c["seed"] + 1,
+                                          poison=False)
+        dargs = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        del q_h, k_h, v_h
+        sec = {"prefill": {}, "decode": {}}
+        ms0, (o0, _) = _timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale), dev, 3)
+        sec["prefill"]["0.0"] = {"ms": ms0, "tflops": fl / (ms0 * 1e-3) / 1e12}
+        dense_bytes = decode_bytes([S], Hq, Hkv, D, cache.max_pages)
+        dms0, (do0, _) = _timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=256), dev, reps, flush)
+        sec["decode"]["0.0"] = {"ms": dms0, "split": 256, "gbs": dense_bytes / (dms0 * 1e-3) / 1e9,
+                                "frac_of_measured_hbm": dense_bytes / (dms0 * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        for lam in (0.1, 0.3):
+            cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+            ms, (o, _, mask) = _timed(lambda: ab.prefill_blasst(q, k, v, lam, causal=True, scale=scale,
+                                                                 skipped_tiles=cnt), dev, 3)
+            vis = mask != 2
+            err = (o.float() - o0.float()).abs()
+            sec["prefill"][str(lam)] = {
+                "ms": ms, "tflops_dense_equiv": fl / (ms * 1e-3) / 1e12,
+                "skipped_frac": float(((mask == 1) & vis).sum().item() / vis.sum().item()),
+                "max_abs_err_vs_dense": float(err.max().item()), "mean_abs_err_vs_dense": float(err.mean().item()),
+                "speedup_vs_dense": ms0 / ms}
+            for split in (2048, 256):
+                for rows in ("group", "head"):
+                    ms, (do, _, dmask) = _timed(
+                        lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split,
+                                                       rows_per_unit=rows), dev, reps, flush)
+                    dvis = dmask != 2
+                    k_b, v_kept = _decode_kept_bytes(dmask, [S], G, D, rows, c["page_size"], cache.max_pages)
+                    v_all = S * Hkv * D * 2
+                    kept_bytes = dense_bytes - v_all + v_kept      # q, o, lse and tables included
+                    sec["decode"][f"{lam}_split{split}_{rows}"] = {
+                        "ms": ms, "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
+                        "bytes_kept": kept_bytes, "v_bytes_saved_frac": 1.0 - v_kept / v_all,
+                        "gbs_on_kept_bytes": kept_bytes / (ms * 1e-3) / 1e9,
+                        "max_abs_err_vs_dense": float((do.float() - do0.float()).abs().max().item()),
+                        "speedup_vs_dense": dms0 / ms}
+        report[name] = sec
+        del q, k, v, dargs
     return report
 
 
