@@ -42,14 +42,17 @@ struct BlScoresSmem {
   static constexpr int kHeadBytes = kDhChunk * D * 2;   // one head's 16 key rows
   static constexpr int kKBytes = HG * kHeadBytes;
   static constexpr int kQBytes = HG * G * D * 2;
-  static constexpr int kStageBytes = (kKBytes + kQBytes + 1023) / 1024 * 1024;
+  static constexpr int kStageBytes = kKBytes;            // a multiple of 1024
   static constexpr int kBlocks = 3;                      // resident CTAs per SM
-  static constexpr int kFit = (233472 / kBlocks - 1024 - 2048) / (kStageBytes + 48);
+  // the query rows of an item sit in one of two buffers of their own (items alternate)
+  static constexpr int kFit = (233472 / kBlocks - 2 * kQBytes - 1024 - 2048) / (kStageBytes + 48);
   static constexpr int kStages = kFit < 6 ? kFit : 6;
   static constexpr int kRing = kStages * kStageBytes;
-  static constexpr int kFull = kRing;
+  static constexpr int kQ = kRing;
+  static constexpr int kFull = kQ + 2 * kQBytes;
   static constexpr int kEmpty = kFull + 8 * kStages;
-  static constexpr int kInfo = kEmpty + 8 * kStages;
+  static constexpr int kQEmpty = kEmpty + 8 * kStages;   // a query buffer was read (count HG)
+  static constexpr int kInfo = kQEmpty + 16;
   static constexpr int kTotal = kInfo + 32 * kStages;
   static constexpr int kDynamic = kTotal + 1024;
   static_assert(kStages >= 2, "ring depth");
@@ -68,6 +71,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kFull);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::kEmpty);
+  uint64_t* qempty = reinterpret_cast<uint64_t*>(smem + L::kQEmpty);
   TileInfo* info = reinterpret_cast<TileInfo*>(smem + L::kInfo);
   __shared__ int abort_flag;
 
@@ -84,6 +88,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], HG);
     }
+    mbar_init(&qempty[0], HG);
+    mbar_init(&qempty[1], HG);
     fence_mbar_init();
   }
   __syncthreads();
@@ -94,6 +100,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
     int slot = 0;
     uint32_t phase = 0;
     uint32_t pending = 0, pending_phase = 0;
+    int qpar = 0;
+    uint32_t q_phase = 0;   // bit b: phase of query buffer b
     bool ok = true;
     long long nx_item = 0;
     int nx_len = 0, nx_win = -1;
@@ -134,6 +142,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
         win_next = e < p.max_pages ? __ldg(&bt_row[e]) : -1;
       }
       const __nv_bfloat16* qsrc = p.q + (size_t(seq) * p.Hq + size_t(grp) * HG * G) * D;
+      // the query buffer of this item must have been read by every consumer for the item before last
+      const int qb = qpar;
+      qpar ^= 1;
+      if (!mbar_wait(&qempty[qb], ((q_phase >> qb) & 1u) ^ 1u, &abort_flag, p.status)) { ok = false; break; }
+      q_phase ^= 1u << qb;
+      uint8_t* qbuf = smem + L::kQ + qb * L::kQBytes;
       for (int t0 = t_begin; t0 < t_end && ok; t0 += kDhChunk) {
         const int e0 = t0 / p.page_size;
         if ((e0 >> 5) != win) {   // a chunk of at most 256 tokens spans at most two windows of 32 pages
@@ -162,7 +176,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
           info[slot] = ti;
           uint8_t* stage = smem + slot * L::kStageBytes;
           mbar_arrive_expect_tx(&full[slot], bytes);
-          if (first) bulk_load(stage + L::kKBytes, qsrc, uint32_t(L::kQBytes), &full[slot]);
+          if (first) bulk_load(qbuf, qsrc, uint32_t(L::kQBytes), &full[slot]);
           if (!ti.bad) tma_load_5d(stage, &tm_k, &full[slot], 0, t0 % p.page_size, 0, grp * HG, page);
         }
         __syncwarp();
@@ -197,6 +211,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
     int no_abort = 0;
     bool ok = true;
     int seq = 0, chunk = 0, grp = 0;
+    int qpar = 0;
     uint32_t qb[KS][2];
     const uint32_t ring_addr = smem_u32(smem);
     float tmax[2] = {neg_inf, neg_inf};   // running row maxima of the current 64-token tile
@@ -207,16 +222,18 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
       if (!mbar_wait(&full[slot], phase, reinterpret_cast<volatile int*>(&no_abort), p.status)) { ok = false; break; }
       const TileInfo ti = info[slot];
       if (ti.flags & 4) break;
-      const uint8_t* stage = smem + slot * L::kStageBytes;
       if (ti.flags & 1) {
         seq = ti.seq; chunk = ti.split; grp = ti.kvh;
-        const uint32_t* qs = reinterpret_cast<const uint32_t*>(stage + L::kKBytes) + warp * G * (D / 2);
+        const uint32_t* qs = reinterpret_cast<const uint32_t*>(smem + L::kQ + qpar * L::kQBytes) + warp * G * (D / 2);
         const bool qv = g < G;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           qb[ks][0] = qv ? qs[g * (D / 2) + ks * 8 + tq] : 0u;
           qb[ks][1] = qv ? qs[g * (D / 2) + ks * 8 + 4 + tq] : 0u;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[qpar]);   // the query buffer may take the item after next
+        qpar ^= 1;
         tmax[0] = tmax[1] = neg_inf;
         cmax[0] = cmax[1] = neg_inf;
       }
@@ -323,7 +340,6 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
                             // that no pipeline wait below starts its clock before pass 1 has finished)
   constexpr int NS = L::kStages;
   constexpr int R = HG * G;                       // query heads (rows) of a group
-  constexpr uint32_t kRows = R == 32 ? 0xffffffffu : ((1u << R) - 1u);
   constexpr uint32_t kUnit = (1u << G) - 1u;      // the rows of one KV head, at bit 0
 
   extern __shared__ uint8_t smem_raw[];
