@@ -410,36 +410,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// 2^x for a pair, on the FMA pipe: x = n + f with n = round(x) (obtained by
-// adding 1.5 * 2^23, which leaves n in the low mantissa bits), f in [-1/2, 1/2];
-// 2^f by a cubic fitted by tests/exp2_poly_fit.py (max relative error 7.7e-5);
-// 2^n applied by adding n to the exponent field. Inputs are clamped to
-// [-126, 64], so masked (-inf) entries come out as ~1e-38.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99992755f, c1 = 0.69325161f, c2 = 0.24261538f, c3 = 0.055222615f;
-  x0 = fminf(fmaxf(x0, -126.f), 64.f);
-  x1 = fminf(fmaxf(x1, -126.f), 64.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t shift = f2_pack(kShift, kShift);
-  const uint64_t t = f2_add(x, shift);
-  const uint64_t n = f2_sub(t, shift);
-  const uint64_t f = f2_sub(x, n);
-  uint64_t p = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
-  p = f2_fma(p, f, f2_pack(c1, c1));
-  p = f2_fma(p, f, f2_pack(c0, c0));
-  float t0, t1, p0, p1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(p, p0, p1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
 
 }  // namespace attn
 

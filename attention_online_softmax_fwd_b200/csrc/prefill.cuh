@@ -401,6 +401,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_smem;
 
+  // The CTA's items: round r takes item r * grid + b, with the CTA order b
+  // reversed on odd rounds (a snake), so that the CTAs that take the longer
+  // item of one round take the shorter of the next: with items in decreasing
+  // causal length, every CTA ends within about one tile of the others.
+  auto pf_item_of = [&](int round) {
+    const int b = (round & 1) ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x);
+    return round * int(gridDim.x) + b;
+  };
   // Item decode shared by all roles: longest causal blocks first; the G query
   // heads of one KV head are adjacent so their K/V tiles are reused from L2.
   auto item_coords = [&](int item, int& qb, int& b, int& hq) {
@@ -452,7 +460,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t qe_bits = 3u;
       uint32_t pend_mask = 0, pend_ph = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+      for (int round = 0, item = pf_item_of(0); item < p.num_items && ok; item = pf_item_of(++round)) {
         int qb, b, hq;
         item_coords(item, qb, b, hq);
         const int kvh = hq / (p.Hq / p.Hkv);
@@ -524,7 +532,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int pend_tag0 = 0, pend_tag1 = 0;   // SKIP: votes of a V tile loaded without its decision
         int gstep = 0;          // ring steps of this CTA (for the test-only withheld step)
         bool ok = true;
-        for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+        for (int round = 0, item = pf_item_of(0); item < p.num_items && ok; item = pf_item_of(++round)) {
           int qb, b, hq;
           item_coords(item, qb, b, hq);
           const int kvh = hq / (p.Hq / p.Hkv);
@@ -635,7 +643,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int seq = 0;              // P V tiles of this query tile so far (skip-vote sequence)
         bool ok = true;
 
-        for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+        for (int round = 0, item = pf_item_of(0); item < p.num_items && ok; item = pf_item_of(++round)) {
           int qb, b, hq;
           item_coords(item, qb, b, hq);
           const int off = seq_offset(b, false);
@@ -723,7 +731,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int seq = 0;   // K/V tiles of this query tile so far (skip-vote sequence)
     bool ok = true;
 
-    for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
+    for (int round = 0, item = pf_item_of(0); item < p.num_items && ok; item = pf_item_of(++round)) {
       int qb, b, hq;
       item_coords(item, qb, b, hq);
       const int off = seq_offset(b, x == 0 && t == 0);
