@@ -130,16 +130,16 @@ int encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int D, 
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
 
-template <int D, bool CAUSAL, bool SKIP, bool PAGED = false>
+template <int D, bool CAUSAL, bool SKIP, bool PAGED = false, bool DBG = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tvh,
                    const PrefillParams& p, int sms, cudaStream_t stream) {
-  auto kernel = prefill_kernel<D, CAUSAL, SKIP, PAGED>;
+  auto kernel = prefill_kernel<D, CAUSAL, SKIP, PAGED, DBG>;
   constexpr int smem = PrefillSmem<D>::kDynamic;
   // The kernel moves registers between warpgroups with setmaxnreg; the block's
   // launch allocation must cover the split or the increase would never return
   // (checked with the shared-memory limit, once per device).
-  if (int st = set_smem_once<prefill_kernel<D, CAUSAL, SKIP, PAGED>>(smem, (kPfRegPoolNeeded + kPfThreads - 1) /
-                                                                            kPfThreads))
+  if (int st = set_smem_once<prefill_kernel<D, CAUSAL, SKIP, PAGED, DBG>>(
+          smem, (kPfRegPoolNeeded + kPfThreads - 1) / kPfThreads))
     return st;
   const long long grid = p.num_items < sms ? p.num_items : sms;
   kernel<<<dim3(unsigned(grid)), dim3(kPfThreads), smem, stream>>>(tq, tk, tv, tvh, p);
@@ -201,6 +201,13 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the mask and the count need the decision path
   const bool use_skip = blasst && (lambda > 0.f || skip_mask != nullptr || skipped_tiles != nullptr);
+  if (dbg.withhold_step >= 0 || dbg.wait_ns != kWaitLimitNs) {   // the test entry point (dense only)
+    if (D == 128)
+      return causal ? launch_prefill<128, true, false, false, true>(tq, tk, tv, tvh, p, sms, s)
+                    : launch_prefill<128, false, false, false, true>(tq, tk, tv, tvh, p, sms, s);
+    return causal ? launch_prefill<64, true, false, false, true>(tq, tk, tv, tvh, p, sms, s)
+                  : launch_prefill<64, false, false, false, true>(tq, tk, tv, tvh, p, sms, s);
+  }
   if (D == 128)
     return use_skip ? dispatch_prefill_causal<128, true>(causal != 0, tq, tk, tv, tvh, p, sms, s)
                     : dispatch_prefill_causal<128, false>(causal != 0, tq, tk, tv, tvh, p, sms, s);

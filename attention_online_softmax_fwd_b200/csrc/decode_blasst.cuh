@@ -415,11 +415,19 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
 #pragma unroll
       for (int i = 0; i < kBlChunkTiles; ++i)
         tm[i] = (lane < R && i < nt) ? p.ws_tmax[row_base * p.max_tiles + ta + i] : neg_inf;
-      // running maximum at the chunk start: the maxima of the split's earlier chunks
+      // running maximum at the chunk start: the maxima of the split's earlier chunks, sixteen
+      // loads in flight at a time (a chain of dependent loads would cost one L2 round trip each)
       float m = neg_inf;
-      if (lane < R) {
+      {
         const int j0 = (t_begin / p.split_tokens) * (p.split_tokens / C);
-        for (int j = j0; j < chunk; ++j) m = fmaxf(m, p.ws_cmax[row_base * p.max_chunks + j]);
+        const float* cm = p.ws_cmax + row_base * p.max_chunks;
+        for (int jb = j0; jb < chunk; jb += 16) {
+          float v[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[u] = (lane < R && jb + u < chunk) ? cm[jb + u] : neg_inf;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) m = fmaxf(m, v[u]);
+        }
       }
       uint32_t keep_t[kBlChunkTiles];
       float mref = neg_inf;

@@ -351,7 +351,10 @@ __device__ __forceinline__ int pf_count_skipped(const PrefillParams& p, int jt, 
 // {D, Hkv, page_size, P} with 16-slot boxes).
 // SKIP: tm_vh maps V with boxes of 64 rows (one 64-key half of a tile), so that
 // the producer loads only the halves that one of the two query tiles keeps.
-template <int D, bool CAUSAL, bool SKIP, bool PAGED = false>
+// DBG (the test entry point only): the producer's and issuers' wait limit comes
+// from p.wait_ns and the producer leaves out ring step p.withhold_step; every
+// other instantiation waits up to kWaitLimitNs and withholds nothing.
+template <int D, bool CAUSAL, bool SKIP, bool PAGED = false, bool DBG = false>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_vh,
@@ -360,6 +363,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   constexpr int NS = L::kStages;
   constexpr int kTmemCols = 512;
   constexpr int kLead = 2;   // K tiles loaded before the first V (pf_ring_step)
+  const unsigned long long wait_lim = DBG ? p.wait_ns : kWaitLimitNs;
 
 
   extern __shared__ uint8_t smem_raw[];
@@ -472,7 +476,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if ((x == 0 ? rows0 : rows1) == 0 || !ok) continue;
           int w = 1;
           if (lane == 0)
-            w = mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status, p.wait_ns) ? 1 : 0;
+            w = mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status, wait_lim) ? 1 : 0;
           if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; continue; }
           qe_bits ^= 1u << x;
           if (lane == 0) {
@@ -500,7 +504,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           const int entry = (tile & 1) ? entry_odd : entry_even;
           int w = 1;
-          if (lane == 0) w = mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status, p.wait_ns) ? 1 : 0;
+          if (lane == 0) w = mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status, wait_lim) ? 1 : 0;
           if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
           if (lane == 0) mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
           if (lane < kPfKeys / 16)
@@ -543,7 +547,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if ((x == 0 ? rows0 : rows1) == 0 || !ok) continue;
-            if (!mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status, p.wait_ns)) {
+            if (!mbar_wait(&bars[L::bQEmpty + x], (qe_bits >> x) & 1u, abort_flag, p.status, wait_lim)) {
               ok = false;
               continue;
             }
@@ -574,13 +578,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 } else if (pend_tag0 | pend_tag1) {
                   // the previous tile's votes (loaded at once): in by now, since Q K^T of this tile,
                   // issued after they were cast, has completed
-                  const int d = pf_dropped_by_both(votes, pend_tag0, pend_tag1, abort_flag, p.status, p.wait_ns);
+                  const int d = pf_dropped_by_both(votes, pend_tag0, pend_tag1, abort_flag, p.status, wait_lim);
                   if (d < 0) { ok = false; break; }
                   prev_dropped = d == 3;
                 }
                 pend_tag0 = pend_tag1 = 0;
                 if (prev_dropped) {
-                  const int dropped = pf_dropped_by_both(votes, tag0, tag1, abort_flag, p.status, p.wait_ns);
+                  const int dropped = pf_dropped_by_both(votes, tag0, tag1, abort_flag, p.status, wait_lim);
                   if (dropped < 0) { ok = false; break; }
                   halves = ~dropped & 3;
                   prev_dropped = dropped == 3;
@@ -590,11 +594,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
               }
             }
-            if (!mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status, p.wait_ns)) {
+            if (!mbar_wait(&bars[L::bKVEmpty + slot], phase ^ 1u, abort_flag, p.status, wait_lim)) {
               ok = false;
               break;
             }
-            if (gstep++ != p.withhold_step) {
+            if (!DBG || gstep++ != p.withhold_step) {
               uint8_t* dst = smem + L::kRing + slot * L::kTileBytes;
               if (halves == 3) {
                 mbar_arrive_expect_tx(&bars[L::bKVFull + slot], L::kTileBytes);
@@ -651,7 +655,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const int n = max(tile_nkv(qb, 0, rows0, off), tile_nkv(qb, 1, rows1, off));
           const int nkv = tile_nkv(qb, x, x == 0 ? rows0 : rows1, off);
           if (nkv > 0) {
-            if (!mbar_wait(&bars[L::bQFull + x], qf_ph, abort_flag, p.status, p.wait_ns)) break;
+            if (!mbar_wait(&bars[L::bQFull + x], qf_ph, abort_flag, p.status, wait_lim)) break;
             qf_ph ^= 1u;
           }
           bool pv_started = false;  // a P V product was issued for this tile in this item
@@ -663,12 +667,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int cur = slot;
             const uint32_t cph = phase;
             if (++slot == NS) { slot = 0; phase ^= 1u; }
-            if (!mbar_wait(&bars[L::bKVFull + cur], cph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
+            if (!mbar_wait(&bars[L::bKVFull + cur], cph, abort_flag, p.status, wait_lim)) { ok = false; break; }
             tc_fence_after();
             if (is_k && tile < nkv) {
               // S_x(tile) = Q_x K_tile^T, once the softmax has copied out S_x(tile - 1)
               if (qk_started) {
-                if (!mbar_wait(&bars[L::bSFree + x], sfree_ph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
+                if (!mbar_wait(&bars[L::bSFree + x], sfree_ph, abort_flag, p.status, wait_lim)) { ok = false; break; }
                 sfree_ph ^= 1u;
                 tc_fence_after();
               }
@@ -679,20 +683,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (tile + 1 == nkv) umma_commit(&bars[L::bQEmpty + x]);   // last Q K^T of this tile
             } else if (!is_k && tile < nkv) {
               // O_x += P_x(tile) V_tile
-              if (!mbar_wait(&bars[L::bPFull + x], pf_ph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
+              if (!mbar_wait(&bars[L::bPFull + x], pf_ph, abort_flag, p.status, wait_lim)) { ok = false; break; }
               pf_ph ^= 1u;
               tc_fence_after();
               int skip_halves = 0;
               if constexpr (SKIP) {
                 // every softmax warp voted before arriving on P_full
                 ++seq;
-                skip_halves = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, abort_flag, p.status, p.wait_ns);
+                skip_halves = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, abort_flag, p.status, wait_lim);
                 if (skip_halves < 0) { ok = false; break; }
               }
               if (skip_halves != 3) {
                 if (!pv_started) {
                   // first P V of this item: the previous item's epilogue must have read O_x
-                  if (!mbar_wait(&bars[L::bOEmpty + x], oe_ph, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
+                  if (!mbar_wait(&bars[L::bOEmpty + x], oe_ph, abort_flag, p.status, wait_lim)) { ok = false; break; }
                   oe_ph ^= 1u;
                   tc_fence_after();
                 }

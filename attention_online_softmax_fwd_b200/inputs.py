@@ -133,6 +133,26 @@ def paged_from_contiguous(q_last, k, v, page_size, seed, poison=True):
                       torch.tensor([k.shape[1]], dtype=torch.int32), page_size)
 
 
+def peaked_decode_batch(num_seqs, Hq, Hkv, L, D, seed, amp=12.0, period=None, page_size=16, poison=False):
+    """A decode batch of ``num_seqs`` sequences of L tokens whose scores are
+    peaked like peaked_prefill_inputs: one seeded unit vector u, amp*u added to
+    every ``period``-th key of each sequence (key 0 only when period is None) and
+    to every query. K/V ~ N(0, 1) otherwise; paged by a seeded permutation."""
+    g = torch.Generator().manual_seed(seed)
+    u = _randn(g, (D,))
+    u = u / u.norm()
+    q = (_randn(g, (num_seqs, Hq, D)) + amp * u).to(torch.bfloat16)
+    step = L if period is None else period
+    k_seqs, v_seqs = [], []
+    for _ in range(num_seqs):
+        k = _randn(g, (L, Hkv, D))
+        k[::step] += amp * u
+        k_seqs.append(k.to(torch.bfloat16))
+        v_seqs.append(_randn(g, (L, Hkv, D)).to(torch.bfloat16))
+    k_pool, v_pool, bt = page_sequences(k_seqs, v_seqs, page_size, g, 0.1, poison)
+    return PagedCache(q, k_pool, v_pool, bt, torch.tensor([L] * num_seqs, dtype=torch.int32), page_size)
+
+
 @dataclass
 class PagedPrefill:
     q: torch.Tensor            # [B, Sq, Hq, D] bf16: queries of the Sq newest tokens

@@ -590,6 +590,31 @@ def blasst_long_context_report(dev, peaks, reps=5):
                         "speedup_vs_dense": dms0 / ms}
         report[name] = sec
         del q, k, v, dargs
+
+    # The same dominant-key pattern over a batch of 8 sequences of 16384 tokens (537 MB of K/V):
+    # enough bytes that the decode is bound by HBM rather than by latency, so that the V rows the
+    # skip does not read show up in the time.
+    cache = gen.peaked_decode_batch(8, Hq, Hkv, 16384, D, c["seed"] + 9, amp=12.0, page_size=c["page_size"])
+    dargs = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    lens = [16384] * 8
+    dense_bytes = decode_bytes(lens, Hq, Hkv, D, cache.max_pages)
+    dms0, (do0, _) = _timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=256), dev, reps, flush)
+    batch = {"workload": "8 sequences x 16384 tokens, 12u on key 0 of each and on every query, Hq32 Hkv8 D128",
+             "0.0": {"ms": dms0, "split": 256, "gbs": dense_bytes / (dms0 * 1e-3) / 1e9}}
+    for lam in (0.1, 0.3):
+        for rows in ("group", "head"):
+            ms, (do, _, dmask) = _timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=2048,
+                                                                       rows_per_unit=rows), dev, reps, flush)
+            dvis = dmask != 2
+            k_b, v_kept = _decode_kept_bytes(dmask, lens, G, D, rows, c["page_size"], cache.max_pages)
+            v_all = sum(lens) * Hkv * D * 2
+            kept_bytes = dense_bytes - v_all + v_kept
+            batch[f"{lam}_split2048_{rows}"] = {
+                "ms": ms, "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
+                "v_bytes_saved_frac": 1.0 - v_kept / v_all, "gbs_on_kept_bytes": kept_bytes / (ms * 1e-3) / 1e9,
+                "max_abs_err_vs_dense": float((do.float() - do0.float()).abs().max().item()),
+                "speedup_vs_dense": dms0 / ms}
+    report["dominant_key_decode_batch"] = batch
     return report
 
 

@@ -109,3 +109,18 @@ def test_library_status_word_is_opt_in(cuda_device):
         assert ab.binding.read_device_status(clear=True) == 4
     finally:
         ab.binding.set_library_status(False)
+
+
+def test_decode_blasst_dominant_key_batch(cuda_device):
+    """A batch with one dominant key per sequence (the bench's bandwidth-bound skip
+    workload, at reduced size): per-head decisions at split 2048 against the oracle."""
+    c = gen.peaked_decode_batch(3, 32, 8, 4096, 128, seed=5400, amp=12.0, page_size=16)
+    for rows in ("group", "head"):
+        o, lse, mask, counted, scale = _run(c, cuda_device, 0.3, 2048, rows)
+        o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(c.q, c.k_pages, c.v_pages, c.block_table,
+                                                                c.seq_lens, 16, scale, 0.3, 2048, rows_per_unit=rows)
+        st = compare_blasst(o, lse, mask, o_ref, lse_ref, m_ref, margin,
+                            lambda m: orc.decode_paged_with_skip_mask(c.q, c.k_pages, c.v_pages, c.block_table,
+                                                                      c.seq_lens, 16, scale, m, rows_per_unit=rows),
+                            label=f"dominant batch {rows}")
+        assert st["skipped"] > 0 and counted == st["skipped_gpu"]
