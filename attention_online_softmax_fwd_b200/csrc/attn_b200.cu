@@ -262,7 +262,7 @@ bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0
 //   [header: two work-ticket counters][partial O [N][max_chunks][Hq][D]][partial lse [N][max_chunks][Hq]]
 //   [scores [N][Hq][tok64]][tile maxima [N][Hq][max_tiles]][chunk maxima [N][Hq][max_chunks]]
 // A work item covers chunk_tokens tokens: the largest of 256, 192, 128, 64 that divides split_tokens (so
-// no chunk straddles a decision split), halved down to 64 while the batch gives fewer than 8192
+// no chunk straddles a decision split), halved down to 64 while the batch gives fewer than 32768
 // (sequence, query head, chunk) triples, so that a few long sequences still fill the GPU.
 struct BlasstLayout {
   int chunk = 0, max_chunks = 0, max_tiles = 0, tok64 = 0;
@@ -279,7 +279,7 @@ bool blasst_layout(int num_seqs, int Hq, int D, int max_pages, int page_size, in
   for (int c : {256, 192, 128}) {
     if (split_tokens % c == 0) { C = c; break; }
   }
-  while (C % 128 == 0 && (long long)num_seqs * Hq * ((cap + C - 1) / C) < 8192) C /= 2;
+  while (C % 128 == 0 && (long long)num_seqs * Hq * ((cap + C - 1) / C) < 32768) C /= 2;
   L->chunk = C;
   L->max_chunks = int((cap + C - 1) / C);
   L->max_tiles = int((cap + 63) / 64);

@@ -378,8 +378,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
     uint32_t phase = 0;
     uint32_t pending = 0, pending_phase = 0;
     bool ok = true;
+    // The next item (ticket), its length and first block-table window, and the maxima its
+    // decisions need -- its tiles' row maxima and the first sixteen chunk maxima of its split
+    // before it -- are all loaded one item ahead, so that an item starts without a round trip.
+    // Lane r < R stands for group row r (query head grp * R + r).
     long long nx_item = 0;
     int nx_len = 0, nx_win = -1;
+    float nx_tm[kBlChunkTiles];
+    float nx_cm[16];
     auto fetch_next = [&]() {
       long long t = 0;
       if (lane == 0) t = atomicAdd(ticket_counter, 1);
@@ -391,6 +397,15 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
         nx_len = __ldg(&p.seq_lens[sq]);
         const int e = (((ch * C) / p.page_size) & ~31) + lane;
         nx_win = e < p.max_pages ? __ldg(&p.block_table[size_t(sq) * p.max_pages + e]) : -1;
+        const size_t rb = size_t(sq) * p.Hq + (lane < R ? gr * R + lane : 0);
+        const int ta = ch * C / kDecTile;
+#pragma unroll
+        for (int i = 0; i < kBlChunkTiles; ++i)   // tiles past the sequence end are read, never used
+          nx_tm[i] = (lane < R && ta + i < p.max_tiles) ? p.ws_tmax[rb * p.max_tiles + ta + i] : neg_inf;
+        const int j0 = (ch * C / p.split_tokens) * (p.split_tokens / C);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          nx_cm[u] = (lane < R && j0 + u < ch) ? p.ws_cmax[rb * p.max_chunks + j0 + u] : neg_inf;
       }
     };
     fetch_next();
@@ -399,6 +414,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
       if (item >= num_items) break;
       int len = nx_len;
       int win_cur = nx_win;
+      float tm[kBlChunkTiles];
+      float m = neg_inf;   // running maximum at the chunk start: the split's earlier chunks' maxima
+#pragma unroll
+      for (int i = 0; i < kBlChunkTiles; ++i) tm[i] = nx_tm[i];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) m = fmaxf(m, nx_cm[u]);
       fetch_next();
       int seq, chunk, grp;
       dh_item_coords(item, p.num_seqs, n_groups, seq, chunk, grp);
@@ -407,19 +428,16 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
       if (t_begin >= len) continue;
       const int t_end = min(t_begin + C, len);
 
-      // ---- decisions of the chunk's tiles; lane r < R is group row r (query head grp * R + r)
+      // ---- decisions of the chunk's tiles
       const int hq = grp * R + lane;
       const size_t row_base = (size_t(seq) * p.Hq + (lane < R ? hq : 0));
-      float tm[kBlChunkTiles];
-      const int ta = t_begin / kDecTile, nt = (t_end - t_begin + kDecTile - 1) / kDecTile;
+      const int nt = (t_end - t_begin + kDecTile - 1) / kDecTile;
 #pragma unroll
       for (int i = 0; i < kBlChunkTiles; ++i)
-        tm[i] = (lane < R && i < nt) ? p.ws_tmax[row_base * p.max_tiles + ta + i] : neg_inf;
-      // running maximum at the chunk start: the maxima of the split's earlier chunks, sixteen
-      // loads in flight at a time (a chain of dependent loads would cost one L2 round trip each)
-      float m = neg_inf;
+        if (i >= nt) tm[i] = neg_inf;
       {
-        const int j0 = (t_begin / p.split_tokens) * (p.split_tokens / C);
+        // chunk maxima beyond the first sixteen of the split (splits longer than 16 chunks)
+        const int j0 = (t_begin / p.split_tokens) * (p.split_tokens / C) + 16;
         const float* cm = p.ws_cmax + row_base * p.max_chunks;
         for (int jb = j0; jb < chunk; jb += 16) {
           float v[16];
@@ -437,7 +455,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
       for (int i = 0; i < kBlChunkTiles; ++i) {
         keep_t[i] = 0;
         if (i >= nt) continue;
-        const int t = ta + i;
+        const int t = t_begin / kDecTile + i;
         if ((t * kDecTile) % p.split_tokens == 0) m = neg_inf;   // a decision split starts with this tile
         const float T = tm[i];
         // the rule for one row: no visible score in the tile, or a finite running maximum that the

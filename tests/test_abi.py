@@ -105,7 +105,7 @@ def _blasst_layout(n, hq, d, mp, ps, sp):
     """The tile-skip workspace as the header documents it (chunk choice included)."""
     cap = mp * ps
     c = next((x for x in (256, 192, 128) if sp % x == 0), 64)
-    while c % 128 == 0 and n * hq * -(-cap // c) < 8192:
+    while c % 128 == 0 and n * hq * -(-cap // c) < 32768:
         c //= 2
     chunks, tiles = -(-cap // c), -(-cap // 64)
     r256 = lambda x: -(-x // 256) * 256
