@@ -48,6 +48,7 @@ SIGNATURES = {
     "attn_prefill_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
     "attn_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_blasst_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "attn_decode_skip_passes": (_I, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P, _P,
                                _P, _SZ, _P, _P, _P, _P]),
     "attn_decode_paged_blasst_heads": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _P,
@@ -235,6 +236,11 @@ def prefill_blasst(q, k, v, lam: float, causal: bool = True, scale: float | None
 def decode_workspace_bytes(num_seqs, Hq, D, max_pages, page_size, split_tokens) -> int:
     """Workspace of the dense decode."""
     return int(load_library().attn_decode_workspace_bytes(num_seqs, Hq, D, max_pages, page_size, split_tokens))
+
+
+def decode_skip_passes(num_seqs, Hq, Hkv, max_pages, page_size, split_tokens) -> int:
+    """Passes over K of the tile-skip decode for these sizes (1 or 2; 0 if rejected)."""
+    return int(load_library().attn_decode_skip_passes(num_seqs, Hq, Hkv, max_pages, page_size, split_tokens))
 
 
 def decode_blasst_workspace_bytes(num_seqs, Hq, D, max_pages, page_size, split_tokens) -> int:

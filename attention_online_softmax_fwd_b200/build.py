@@ -11,8 +11,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn_b200.so")
 SOURCES = ["attn_b200.cu"]
-DEPS = ["attn_b200.cu", "common.cuh", "decode.cuh", "decode_blasst.cuh", "decode_heads.cuh", "kv_append.cuh",
-        "prefill.cuh"]
+DEPS = ["attn_b200.cu", "common.cuh", "decode.cuh", "decode_blasst.cuh", "decode_gate.cuh", "decode_heads.cuh",
+        "kv_append.cuh", "prefill.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -13,6 +13,7 @@
 #include "decode.cuh"
 #include "decode_heads.cuh"
 #include "decode_blasst.cuh"
+#include "decode_gate.cuh"
 #include "kv_append.cuh"
 #include "prefill.cuh"
 
@@ -439,6 +440,52 @@ int dispatch_blasst(int G, int hg, bool per_head, const CUtensorMap& tk, const C
                   : dispatch_blasst_g<D, 1, false>(G, tk, tvg, tvh, p, tickets, sms, s);
 }
 
+// Single-pass tile-skip decode over the splits, then the merge of the split partials.
+template <int D, int G, int HG, bool PER_HEAD>
+int launch_gate(const CUtensorMap& tk, const CUtensorMap& tvh, const DecodeParams& p, int* ticket_counter, int sms,
+                cudaStream_t stream) {
+  using L = GateSmem<D, G, HG>;
+  if (int st = set_smem_once<decode_gate_kernel<D, G, HG, PER_HEAD>>(L::kDynamic)) return st;
+  const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
+  const long long slots = (long long)sms * L::kBlocks;
+  decode_gate_kernel<D, G, HG, PER_HEAD><<<dim3(unsigned(items < slots ? items : slots)), dim3((HG + 1) * 32),
+                                           L::kDynamic, stream>>>(tk, tvh, p, ticket_counter);
+  if (int st = launch_status()) return st;
+  return launch_merge<D>(p, stream);
+}
+
+template <int D, int HG, bool PER_HEAD>
+int dispatch_gate_g(int G, const CUtensorMap& tk, const CUtensorMap& tvh, const DecodeParams& p, int* tickets,
+                    int sms, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_gate<D, 1, HG, PER_HEAD>(tk, tvh, p, tickets, sms, s);
+    case 2: return launch_gate<D, 2, HG, PER_HEAD>(tk, tvh, p, tickets, sms, s);
+    case 4: return launch_gate<D, 4, HG, PER_HEAD>(tk, tvh, p, tickets, sms, s);
+    case 8: return launch_gate<D, 8, HG, PER_HEAD>(tk, tvh, p, tickets, sms, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+template <int D>
+int dispatch_gate(int G, int hg, bool per_head, const CUtensorMap& tk, const CUtensorMap& tvh, const DecodeParams& p,
+                  int* tickets, int sms, cudaStream_t s) {
+  if (hg == 2)
+    return per_head ? dispatch_gate_g<D, 2, true>(G, tk, tvh, p, tickets, sms, s)
+                    : dispatch_gate_g<D, 2, false>(G, tk, tvh, p, tickets, sms, s);
+  return per_head ? dispatch_gate_g<D, 1, true>(G, tk, tvh, p, tickets, sms, s)
+                  : dispatch_gate_g<D, 1, false>(G, tk, tvh, p, tickets, sms, s);
+}
+
+// The tile-skip decode for Hq / Hkv <= 8 runs in one pass over the splits when the batch has
+// at least this many (sequence, KV head, split) triples -- enough split items to keep every SM
+// streaming -- and in two passes over chunks of the splits otherwise.
+constexpr long long kGateMinKvSplits = 2048;
+
+int skip_passes(int num_seqs, int Hq, int Hkv, long long max_splits) {
+  if (Hq / Hkv > 8) return 1;
+  return (long long)num_seqs * Hkv * max_splits >= kGateMinKvSplits ? 1 : 2;
+}
+
 // FP8 cache (D = 128): groups of 4 KV heads for G <= 8; G = 16 takes groups of hg (8 or 4)
 int dispatch_decode_heads_fp8(int G, int hg, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                               int* ctr, int sms, cudaStream_t s) {
@@ -470,6 +517,15 @@ const char* attn_status_string(int status) {
 }
 
 int attn_abi_version(void) { return 2; }
+
+int attn_decode_skip_passes(int num_seqs, int Hq, int Hkv, int max_pages_per_seq, int page_size, int split_tokens) {
+  if (num_seqs < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages_per_seq < 1 || !valid_page_size(page_size) ||
+      split_tokens < 64 || split_tokens % 64 != 0)
+    return 0;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return 0;
+  return skip_passes(num_seqs, Hq, Hkv, max_splits_of(max_pages_per_seq, page_size, split_tokens));
+}
 
 int attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S,
                  int D, int causal, float scale, void* stream) {
@@ -639,6 +695,18 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
   // {64 columns, token, 64-column half, head, page}: a head's 16 tokens land as [half][token][64]
   const uint64_t hdims[5] = {64, uint64_t(page_size), uint64_t(D / 64), uint64_t(Hkv), uint64_t(num_pages)};
   const uint64_t hstrides[4] = {uint64_t(Hkv) * D * 2, 128, uint64_t(D) * 2, uint64_t(page_size) * Hkv * D * 2};
+  if (use_skip && G <= 8 && skip_passes(num_seqs, Hq, Hkv, ms) == 1) {
+    // one pass over the splits, groups of 2 KV heads (of 1 when Hkv is odd); V rows per head
+    const int ghg = Hkv % 2 == 0 ? 2 : 1;
+    const uint32_t gbox[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), uint32_t(ghg), 1};
+    const uint32_t box1[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), 1, 1};
+    CUtensorMap gk, gvh;
+    if (int st = encode_map5(&gk, k_pages, hdims, hstrides, gbox)) return st;
+    if (int st = encode_map5(&gvh, v_pages, hdims, hstrides, box1)) return st;
+    if (cudaMemsetAsync(ticket_counter, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (D == 128) return dispatch_gate<128>(G, ghg, per_head, gk, gvh, p, ticket_counter, sms, s);
+    return dispatch_gate<64>(G, ghg, per_head, gk, gvh, p, ticket_counter, sms, s);
+  }
   if (use_skip && G <= 8) {
     // two passes over groups of 4 KV heads (of 1 when Hkv is not a multiple of 4)
     const int bhg = Hkv % 4 == 0 ? 4 : 1;

@@ -186,17 +186,33 @@ size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_pe
 /*
  * attn_decode_blasst_workspace_bytes -- scratch needed by attn_decode_paged and
  * attn_decode_paged_blasst_heads on their tile-skip path (lambda > 0, a
- * skip_mask or a skipped_tiles counter, or the per-head entry point). That path
- * runs in two passes: the first computes the scaled scores of every cached
- * token and query head, and the row maxima of every 64-token tile and of every
- * work chunk; the second derives the decisions from the maxima and reads V only
- * for kept tiles. The workspace holds the scores (fp32
- * [num_seqs][Hq][padded tokens]), the maxima, and one partial (O, LSE) per
- * (sequence, query head, chunk); a chunk is at most 256 tokens and divides
- * split_tokens. Returns 0 for invalid arguments or an overflowing size.
+ * skip_mask or a skipped_tiles counter, or the per-head entry point). With
+ * Hq / Hkv <= 8 that path runs in one or two passes over K, as
+ * attn_decode_skip_passes says. One pass: each (sequence, KV head, split) is
+ * walked in token order and a tile's V rows are read after its decision. Two
+ * passes, for batches with too few splits to fill the GPU: the first computes
+ * the scaled scores of every cached token and query head, and the row maxima
+ * of every 64-token tile and of every work chunk; the second derives the
+ * decisions from the maxima and reads V only for kept tiles. The size covers
+ * both: the scores (fp32 [num_seqs][Hq][padded tokens]), the maxima, and one
+ * partial (O, LSE) per (sequence, query head, chunk); a chunk is at most 256
+ * tokens and divides split_tokens. Returns 0 for invalid arguments or an
+ * overflowing size.
  */
 size_t attn_decode_blasst_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq,
                                           int page_size, int split_tokens);
+
+/*
+ * attn_decode_skip_passes -- how many passes over the cached K the tile-skip
+ * decode makes for these sizes (host arithmetic only, nothing is launched):
+ * 1 when Hq / Hkv = 16 (a one-pass kernel that also reads the skipped tiles'
+ * V rows) or when num_seqs * Hkv * max_splits >= 2048, with max_splits =
+ * ceil(max_pages_per_seq * page_size / split_tokens); 2 otherwise. Both give
+ * the same decisions; the results agree up to the rounding of a different
+ * summation order. Returns 0 for arguments attn_decode_paged would reject.
+ */
+int attn_decode_skip_passes(int num_seqs, int Hq, int Hkv, int max_pages_per_seq, int page_size,
+                            int split_tokens);
 
 /*
  * attn_decode_paged -- single-token decode over a paged KV cache (split-KV
