@@ -305,28 +305,30 @@ bool blasst_layout(int num_seqs, int Hq, int D, int max_pages, int page_size, in
   return true;
 }
 
-// One CTA per (sequence, query head); a no-op for sequences of one split. Launched
-// as a programmatic dependent of the split kernel: it is scheduled while the split
-// kernel's last CTAs run and waits (griddepcontrol.wait) for that grid to finish
-// and its writes to be visible before it reads the partials.
-// Sixteen warps per (sequence, head) when a row has more than 64 partials (long
-// sequences at small splits), four otherwise.
+// One CTA per (sequence, query head); a no-op for sequences of one split.
+// Launched as a programmatic dependent of the split kernel: it is scheduled
+// while the split kernel's last CTAs run and waits (griddepcontrol.wait) for
+// that grid to finish and its writes to be visible before it reads the partials.
+// A row with more than 64 partials (long sequences at small splits) takes
+// sixteen warps on each of D / 32 CTAs, one per 32 head dimensions; four warps on
+// one CTA otherwise.
 template <int D>
 int launch_merge(const DecodeParams& p, cudaStream_t stream) {
   const long long pairs = (long long)p.num_seqs * p.Hq;
   const bool wide = p.max_splits > 64;
+  constexpr int kSlices = D / 32;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(pairs));
+  cfg.gridDim = dim3(unsigned(wide ? pairs * kSlices : pairs));
   cfg.blockDim = dim3((wide ? 16 : 4) * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 16>, p)
-                             : cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 4>, p);
+  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 16, kSlices>, p)
+                             : cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 4, 1>, p);
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   return launch_status();
 }
@@ -356,18 +358,36 @@ int dispatch_decode_g(int G, const CUtensorMap& tk, const CUtensorMap& tv, const
   }
 }
 
+template <int D, int G, int HG, bool F8, int BLOCKS>
+int launch_decode_heads_blocks(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                               int* ticket_counter, int sms, cudaStream_t stream) {
+  using L = DecodeHeadsSmem<D, G, HG, F8, BLOCKS>;
+  auto kernel = decode_heads_kernel<D, G, HG, F8, BLOCKS>;
+  if (int st = set_smem_once<decode_heads_kernel<D, G, HG, F8, BLOCKS>>(L::kDynamic)) return st;
+  const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
+  const long long slots = (long long)sms * L::kBlocks;
+  const long long grid = items < slots ? items : slots;
+  DecodeParams pk = p;
+  pk.static_items = items <= slots ? 1 : 0;   // one item per CTA: no ticket counter to zero
+  if (!pk.static_items && cudaMemsetAsync(ticket_counter, 0, sizeof(int), stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  kernel<<<dim3(unsigned(grid)), dim3((HG + 1) * 32), L::kDynamic, stream>>>(tk, tv, pk, ticket_counter);
+  if (int st = launch_status()) return st;
+  return launch_merge<D>(p, stream);
+}
+
+// A grid of at most two items per SM (few sequences, each with few splits) runs two CTAs
+// per SM with three stages each; anything larger the default residency.
 template <int D, int G, int HG, bool F8 = false>
 int launch_decode_heads(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, int* ticket_counter,
                         int sms, cudaStream_t stream) {
-  auto kernel = decode_heads_kernel<D, G, HG, F8>;
-  constexpr int smem = DecodeHeadsSmem<D, G, HG, F8>::kDynamic;
-  if (int st = set_smem_once<decode_heads_kernel<D, G, HG, F8>>(smem)) return st;
-  const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
-  const long long slots = (long long)sms * DecodeHeadsSmem<D, G, HG, F8>::kBlocks;
-  const long long grid = items < slots ? items : slots;
-  kernel<<<dim3(unsigned(grid)), dim3((HG + 1) * 32), smem, stream>>>(tk, tv, p, ticket_counter);
-  if (int st = launch_status()) return st;
-  return launch_merge<D>(p, stream);
+  constexpr bool kDeep = !F8 && G <= 4;   // the layouts whose default is three CTAs per SM
+  if constexpr (kDeep) {
+    const long long items = (long long)p.max_splits * p.num_seqs * (p.Hkv / HG);
+    if (items <= 2ll * sms)
+      return launch_decode_heads_blocks<D, G, HG, F8, 2>(tk, tv, p, ticket_counter, sms, stream);
+  }
+  return launch_decode_heads_blocks<D, G, HG, F8, 0>(tk, tv, p, ticket_counter, sms, stream);
 }
 
 // groups of 4 KV heads for G <= 8 (several CTAs per SM); G = 16 takes groups of hg (8 or 4)
@@ -637,7 +657,8 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
     return ATTN_ERR_INVALID_ARG;
   if (!aligned4(block_table) || !aligned4(seq_lens) || !aligned4(lse)) return ATTN_ERR_INVALID_ARG;
   if (num_seqs < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if ((long long)num_seqs * Hq > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;   // one merge CTA per (sequence, head)
+  // merge CTAs: one per (sequence, head), or one per 32 of its head dimensions
+  if ((long long)num_seqs * Hq * (D / 32) > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   if (!valid_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
   if (split_tokens < 64 || split_tokens % 64 != 0) return ATTN_ERR_INVALID_ARG;
@@ -737,7 +758,6 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
     CUtensorMap hk, hv;
     if (int st = encode_map5(&hk, k_pages, hdims, hstrides, hbox)) return st;
     if (int st = encode_map5(&hv, v_pages, hdims, hstrides, hbox)) return st;
-    if (cudaMemsetAsync(ticket_counter, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
     if (D == 128) return dispatch_decode_heads<128>(G, hg, hk, hv, p, ticket_counter, sms, s);
     return dispatch_decode_heads<64>(G, hg, hk, hv, p, ticket_counter, sms, s);
   }
@@ -810,7 +830,8 @@ int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_code
     return ATTN_ERR_INVALID_ARG;
   if (!aligned4(block_table) || !aligned4(seq_lens) || !aligned4(lse)) return ATTN_ERR_INVALID_ARG;
   if (num_seqs < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if ((long long)num_seqs * Hq > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;   // one merge CTA per (sequence, head)
+  // merge CTAs: one per (sequence, head), or one per 32 of its head dimensions
+  if ((long long)num_seqs * Hq * (D / 32) > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;
   if (!valid_page_size(page_size) || max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
   if (split_tokens < 64 || split_tokens % 64 != 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
@@ -867,7 +888,6 @@ int attn_decode_paged_fp8(const void* q, const void* k_codes, const void* v_code
                           CU_TENSOR_MAP_DATA_TYPE_UINT8))
     return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ticket_counter, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
   return dispatch_decode_heads_fp8(G, hg, hk, hv, p, ticket_counter, sms, s);
 }
 

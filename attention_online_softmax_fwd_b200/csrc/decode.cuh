@@ -48,6 +48,7 @@ struct DecodeParams {
   float v_scale;      // FP8 cache: V = v_scale * code (the K scale is folded into scale_log2)
   int per_head;       // tile skip decided for each query head alone, not for the KV head's group
   long long num_items;
+  int static_items;   // head-group kernel: at most one item per CTA, item = blockIdx.x (no ticket counter)
   // two-pass tile-skip decode (decode_blasst.cuh); the work items are chunks of
   // chunk_tokens tokens (a divisor of split_tokens), the decision units are splits
   float* ws_s;        // scaled scores (log2 units) [N][Hkv / HG][tok64][HG][G]
@@ -586,23 +587,29 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
 }
 
-// Combine the split partials of one (sequence, query head) per CTA: each
-// partial is a normalised O row (fp32) with its log2-sum-exp; the result is
+// Combine the split partials of one (sequence, query head) per CTA -- or of
+// one of DS slices of its head dimension: each partial is a normalised O row
+// (fp32) with its log2-sum-exp; the result is
 // sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M), M the largest lse_s. Warp w
 // takes splits w, w + W, ... in chunks of kMergeChunk, loading each chunk's
 // lse values and O rows together (one memory round trip per chunk), and keeps a
 // running maximum; the W warps then combine in a fixed order (deterministic).
-// W = 4 serves batches of many sequences; W = 16 puts four times as many
-// partials in flight for the few rows of a long single sequence.
+// W = 4 serves batches of many sequences; W = 16 with one slice per 32 head
+// dimensions puts many partials in flight on many SMs for the few rows of a
+// long single sequence.
 constexpr int kMergeChunk = 8;   // splits per warp in flight
-template <int D, int W = 4>
+template <int D, int W = 4, int DS = 1>
 __global__ void __launch_bounds__(W * 32) decode_merge_kernel(const DecodeParams p) {
+  static_assert((D / 32) % DS == 0, "a slice gives each lane whole floats");
   constexpr int kMergeWarps = W;
-  constexpr int DL = D / 32;   // floats per lane: 4 (D = 128) or 2 (D = 64)
+  constexpr int DW = D / DS;    // head dimensions of this CTA's slice
+  constexpr int DL = DW / 32;   // floats per lane: 4, 2 or 1
   __shared__ float sh_m[kMergeWarps], sh_w[kMergeWarps];
-  __shared__ __align__(16) float sh_acc[kMergeWarps][D];
+  __shared__ __align__(16) float sh_acc[kMergeWarps][DW];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int seq = int(blockIdx.x / unsigned(p.Hq)), hq = int(blockIdx.x % unsigned(p.Hq));
+  const unsigned row = blockIdx.x / unsigned(DS);
+  const int slice = int(blockIdx.x % unsigned(DS));
+  const int seq = int(row / unsigned(p.Hq)), hq = int(row % unsigned(p.Hq));
   const int capacity = p.max_pages * p.page_size;
   // the lengths are inputs, not results of the split kernel: read before waiting for it
   int len = __ldg(&p.seq_lens[seq]);
@@ -611,16 +618,16 @@ __global__ void __launch_bounds__(W * 32) decode_merge_kernel(const DecodeParams
   // every CTA waits for the split kernel (launched as its programmatic dependent), so that this
   // grid never completes before that one
   grid_dependency_wait();
-  __nv_bfloat16* orow = p.o + (size_t(seq) * p.Hq + hq) * D;
+  __nv_bfloat16* orow = p.o + (size_t(seq) * p.Hq + hq) * D + slice * DW;
   const float neg_inf = -__int_as_float(0x7f800000);
   if (n_splits == 1) return;  // written by the split kernel
   if (n_splits == 0) {        // a row the split kernel never writes
-    for (int d = threadIdx.x; d < D; d += blockDim.x) orow[d] = __float2bfloat16_rn(0.f);
-    if (p.lse && threadIdx.x == 0) p.lse[size_t(seq) * p.Hq + hq] = neg_inf;
+    for (int d = threadIdx.x; d < DW; d += blockDim.x) orow[d] = __float2bfloat16_rn(0.f);
+    if (p.lse && slice == 0 && threadIdx.x == 0) p.lse[size_t(seq) * p.Hq + hq] = neg_inf;
     return;
   }
   const float* lse_base = p.ws_lse + size_t(seq) * p.max_splits * p.Hq + hq;
-  const float* o_base = p.ws_o + (size_t(seq) * p.max_splits * p.Hq + hq) * D + lane * DL;
+  const float* o_base = p.ws_o + (size_t(seq) * p.max_splits * p.Hq + hq) * D + slice * DW + lane * DL;
   const size_t o_stride = size_t(p.Hq) * D;   // floats between consecutive splits
   float acc[DL];
 #pragma unroll
@@ -640,9 +647,11 @@ __global__ void __launch_bounds__(W * 32) decode_merge_kernel(const DecodeParams
         if constexpr (DL == 4) {
           const float4 t = *reinterpret_cast<const float4*>(src);
           ov[u][0] = t.x; ov[u][1] = t.y; ov[u][2] = t.z; ov[u][3] = t.w;
-        } else {
+        } else if constexpr (DL == 2) {
           const float2 t = *reinterpret_cast<const float2*>(src);
           ov[u][0] = t.x; ov[u][1] = t.y;
+        } else {
+          ov[u][0] = *src;
         }
       }
     }
@@ -679,13 +688,13 @@ __global__ void __launch_bounds__(W * 32) decode_merge_kernel(const DecodeParams
     wt += f[w] * sh_w[w];
   }
   const float inv = wt > 0.f ? 1.f / wt : 0.f;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+  for (int d = threadIdx.x; d < DW; d += blockDim.x) {
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < kMergeWarps; ++w) v = fmaf(f[w], sh_acc[w][d], v);
     orow[d] = __float2bfloat16_rn(v * inv);
   }
-  if (p.lse && threadIdx.x == 0)
+  if (p.lse && slice == 0 && threadIdx.x == 0)
     p.lse[size_t(seq) * p.Hq + hq] = wt > 0.f ? (mx + __log2f(wt)) * 0.69314718055994531f : neg_inf;
 }
 

@@ -11,12 +11,13 @@
 // transposed products), decides the tile from its row maxima and the split's
 // running maximum (maximum of the earlier tiles' row maxima), and only then asks
 // for the tile's V rows of its own head: one 16-token TMA copy per stage, issued
-// by the warp into one of two tile buffers of its own. A kept tile's P V runs
-// when its buffer is needed again, two kept tiles later, so that each warp keeps
-// two V copies on the way while it scores on; a split's last tiles are finished
-// at the end of the next split's first tile, the warp keeping the split's
-// accumulators until then. Split partials go to the log-sum-exp merge kernel
-// like the dense kernel's.
+// by the warp into a tile buffer of its own (kVBufs of them). A kept tile's P V
+// runs when its buffer is needed again, kVBufs kept tiles later, so that the V
+// copy lands while the warp scores on; a split's last tiles are finished at the
+// end of the next split's first tile, the warp keeping the split's accumulators
+// until then. Split partials go to the log-sum-exp merge kernel like the dense
+// kernel's. One buffer per warp at three CTAs per SM measured faster than two
+// buffers at two CTAs per SM: the stream depth is set by the CTAs' K rings.
 //
 // The two-pass kernels (decode_blasst.cuh) decouple the work items from the
 // decision splits; this one needs enough splits to fill the GPU, and in return

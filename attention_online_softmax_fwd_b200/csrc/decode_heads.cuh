@@ -2,7 +2,8 @@
 //
 // Work item = (split, sequence, group of HG KV heads), handed out in that
 // order (largest splits first) by an atomic ticket counter in the workspace,
-// which the host zeroes before the launch. A stage is 16 tokens of the item:
+// which the host zeroes before the launch; when the grid has a CTA for every
+// item, CTA b takes item b and the counter is not used. A stage is 16 tokens of the item:
 // one TMA copy brings the K rows of all HG heads (a contiguous 16-token x HG-head
 // block of a page) and one the V rows; the tensor map orders heads outside
 // tokens, so each head's 16 rows land as one 4 KB (D = 128) 128-byte-swizzled
@@ -46,12 +47,14 @@ constexpr int kDhChunk = 16;  // tokens per TMA copy (one 16-slot block of a pag
 // tensor) to spread the per-stage costs over more tokens.
 constexpr int kTrBlocks = 3;   // resident CTAs per SM for G <= 4 (registers: 3 x 160 threads x <= 136)
 
-template <int D, int G, int HG, bool F8 = false>
+// BLOCKS = 0: the default residency below; BLOCKS = 2 serves grids of at most two items per
+// SM (a single long sequence), whose CTAs then keep three stages in flight instead of two.
+template <int D, int G, int HG, bool F8 = false, int BLOCKS = 0>
 struct DecodeHeadsSmem {
   static constexpr bool kTr = G <= 8;                            // transposed products
   static constexpr int kHalves = (kTr && F8) ? 2 : 1;            // 16-token copies per tensor per stage
   static constexpr int kTok = kDhChunk * kHalves;                // tokens per stage
-  static constexpr int kBlocks = kTr ? (G <= 4 ? kTrBlocks : 2) : 1;   // resident CTAs per SM
+  static constexpr int kBlocks = BLOCKS > 0 ? BLOCKS : (kTr ? (G <= 4 ? kTrBlocks : 2) : 1);   // CTAs per SM
   static constexpr int kHeadBytes = kDhChunk * D * (F8 ? 1 : 2);   // one head's 16 tokens
   static constexpr int kHalfBytes = HG * kHeadBytes;             // one copy: 16 tokens of the HG heads
   static constexpr int kKVBytes = kHalves * kHalfBytes;          // K (or V) rows of one stage
@@ -89,13 +92,13 @@ __device__ __forceinline__ void dh_item_coords(long long item, int num_seqs, int
   grp = rem % n_groups;
 }
 
-template <int D, int G, int HG, bool F8 = false>
-__global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::kBlocks)
+template <int D, int G, int HG, bool F8 = false, int BLOCKS = 0>
+__global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8, BLOCKS>::kBlocks)
     decode_heads_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeParams p, int* ticket_counter) {
   static_assert(G >= 1 && G <= 16, "query heads per KV head");
   static_assert(!F8 || D == 128, "the FP8 cache layout assumes 128-byte rows");
-  using L = DecodeHeadsSmem<D, G, HG, F8>;
+  using L = DecodeHeadsSmem<D, G, HG, F8, BLOCKS>;
   launch_dependents();   // let the merge kernel be scheduled early; it waits for this grid to finish
   constexpr int NS = L::kStages;
   constexpr int KS = D / 16;
@@ -137,10 +140,16 @@ __global__ void __launch_bounds__((HG + 1) * 32, DecodeHeadsSmem<D, G, HG, F8>::
     // next item (ticket), its length and first block-table window, one item ahead
     long long nx_item = 0;
     int nx_len = 0, nx_win = -1;
+    bool first_fetch = true;
     auto fetch_next = [&]() {
       long long t = 0;
-      if (lane == 0) t = atomicAdd(ticket_counter, 1);
-      t = __shfl_sync(0xffffffffu, t, 0);
+      if (p.static_items) {
+        t = first_fetch ? (long long)blockIdx.x : num_items;
+      } else {
+        if (lane == 0) t = atomicAdd(ticket_counter, 1);
+        t = __shfl_sync(0xffffffffu, t, 0);
+      }
+      first_fetch = false;
       nx_item = t;
       if (t < num_items) {
         int sq, sp, gr;

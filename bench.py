@@ -4,7 +4,8 @@ One step = one causal GQA prefill (B=2, Hq=32, Hkv=8, S=8192, D=128, the shape o
 a Llama-3-8B / Mistral layer) followed by one paged GQA decode (64 sequences,
 lengths uniform in [512, 8192], Hq=32, Hkv=8, D=128, 16-token pages from a
 shared pool in random order). Inputs are seeded synthetic bf16 N(0, 1) data
-resident in HBM. L2 is flushed (a 256 MiB write) before every timed step.
+resident in HBM. L2 is flushed before every timed step (a 256 MiB write, then a 256 MiB read of
+another buffer, so that no dirty line of the flush is written back inside the timed region).
 Kernels are timed with CUDA events on the launching stream.
 
 value = prefill TFLOP/s (algorithmic FLOPs: 4*D per visible (query, key) pair,
@@ -266,7 +267,7 @@ def run_gpu(args, world, rank, local):
     ws = torch.empty(ab.decode_workspace_bytes(dc["N"], dc["Hq"], dc["D"], cache.max_pages, dc["page_size"],
                                                DECODE_SPLIT), dtype=torch.uint8, device=dev)
     scale = gen.attn_scale(D)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def prefill_call():
         ab.prefill(q, k, v, causal=True, scale=scale, out=o, lse=lse)
@@ -276,7 +277,7 @@ def run_gpu(args, world, rank, local):
                         workspace=ws)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         prefill_call()
         decode_call()
     torch.cuda.synchronize()
@@ -288,7 +289,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         ev[i][0].record(stream)
         prefill_call()
         ev[i][1].record(stream)
@@ -332,7 +333,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     e2e_pre, e2e_dec = [], []
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         e0 = torch.cuda.Event(enable_timing=True)
         e2 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -365,7 +366,7 @@ def run_gpu(args, world, rank, local):
             "decode": {"num_seqs": dc["N"], "Hq": dc["Hq"], "Hkv": dc["Hkv"], "D": dc["D"],
                        "page_size": dc["page_size"], "len_range": [dc["len_lo"], dc["len_hi"]],
                        "split_tokens": DECODE_SPLIT, "tokens": int(cache.seq_lens.sum()), "seed": dc["seed"]},
-            "l2": "flushed before every timed step (256 MiB write)",
+            "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer)",
             "parallelism": f"replica x{world}" if world > 1 else "single GPU",
         },
         "prefill": {"ms": pre_ms, "tflops": pre_tfs, "flops_per_launch": fl,
@@ -394,6 +395,7 @@ def run_gpu(args, world, rank, local):
         line["mha_prefill"] = mha_prefill_report(dev, peaks)
     if rank == 0 and world == 1 and not args.no_blasst:
         line["blasst_long_context"] = blasst_long_context_report(dev, peaks)
+        line["decode_skip_nothing_skipped"] = skip_overhead_report(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfs, gbs, secs, desc = oracle_sample(int(args.cpu_heads), 4)
         line["cpu_baseline"] = {"value": tfs, "unit": "TFLOP/s", "cores": cpu_threads()[0], "kind": "oracle",
@@ -427,7 +429,7 @@ def fp8_decode_report(dev, peaks, cache, flush, reps=10):
     torch.cuda.synchronize()
     ts = []
     for _ in range(reps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         call()
@@ -484,13 +486,27 @@ def mha_prefill_report(dev, peaks, reps=20):
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
     scale = gen.attn_scale(D)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     ms = _timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale, out=o, lse=lse), dev, reps, flush)[0]
     fl = prefill_flops(B, Hq, S, D)
     tf = fl / (ms * 1e-3) / 1e12
     return {"workload": "mha_prefill_llama2_7b B4 Hq32 Hkv32 S2048 D128 causal", "kernel": "prefill_kernel<128,causal>",
             "ms": ms, "tflops": tf, "flops_per_launch": fl, "frac_of_measured_bf16": tf / peaks["bf16_tflops"],
             "frac_of_spec_2250": tf / SPEC_PEAKS["bf16_tflops"], "l2": "flushed before every launch"}
+
+
+class L2Flush:
+    """Evicts the timed work's inputs from L2 (126 MB) between timed iterations: writes a
+    256 MiB buffer, then reads another 256 MiB buffer, so that L2 is left holding clean lines
+    of unrelated data and the timed kernels pay no write-back of the flush's own dirty lines."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
 
 
 def _timed(fn, dev, reps, flush=None):
@@ -501,7 +517,7 @@ def _timed(fn, dev, reps, flush=None):
     ts = []
     for _ in range(reps):
         if flush is not None:
-            flush.zero_()
+            flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         out = fn()
@@ -530,23 +546,49 @@ def _decode_kept_bytes(mask, seq_lens, G, D, rows_per_unit, page_size, max_pages
     return sum(L) * kept.shape[1] * D * 2, toks * D * 2    # (K bytes, kept V bytes)
 
 
+def _skip_decode_line(ab, dargs, lam, split, rows, lens, G, D, page_size, max_pages, dense_bytes, dms0, do0,
+                      scale, dev, reps, flush, ws):
+    """One tile-skip decode configuration: timed without the decision mask (a fill kernel
+    the caller would not run), then run once more with it for the statistics."""
+    N, Hq, _ = dargs[0].shape
+    Hkv = dargs[1].shape[2]
+    ms, _ = _timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split, rows_per_unit=rows,
+                                                  skip_mask=False, workspace=ws), dev, reps, flush)
+    do, _, dmask = ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split, rows_per_unit=rows,
+                                          workspace=ws)
+    dvis = dmask != 2
+    _, v_kept = _decode_kept_bytes(dmask, lens, G, D, rows, page_size, max_pages)
+    v_all = sum(lens) * Hkv * D * 2
+    kept_bytes = dense_bytes - v_all + v_kept      # q, o, lse and tables included
+    return {"ms": ms, "passes": ab.binding.decode_skip_passes(N, Hq, Hkv, max_pages, page_size, split),
+            "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
+            "bytes_kept": kept_bytes, "v_bytes_saved_frac": 1.0 - v_kept / v_all,
+            "gbs_on_kept_bytes": kept_bytes / (ms * 1e-3) / 1e9,
+            "max_abs_err_vs_dense": float((do.float() - do0.float()).abs().max().item()),
+            "speedup_vs_dense": dms0 / ms}
+
+
 def blasst_long_context_report(dev, peaks, reps=5):
     """Long-context BLASST workload (B=1, Hq=32, Hkv=8, S=32768, D=128, 64-key tiles,
     lambda in {0, 0.1, 0.3}): prefill, and the decode of the last row over the paged
-    cache at split_tokens = 2048 (the decision split of the workload; 256 as an
-    extra line), for the recipe input (4u on every 64th key) and a single dominant
-    key (12u on key 0). Reports times, skipped fractions, the kept-tile bytes the
-    decode reads, the error against lambda = 0 and the speedup over the dense path
-    (the dense decode at its fastest split, 256)."""
+    cache at split_tokens = 2048 (the decision split of the workload; 256 and one
+    split over the whole sequence as extra lines), for the recipe input (4u on every
+    64th key) and a single dominant key (12u on key 0); then the dominant-key pattern
+    over a batch of 8 x 16384 tokens. Reports times, the number of passes over K,
+    skipped fractions, the kept-tile bytes the decode reads, the error against
+    lambda = 0 and the speedup over the dense path (the dense decode at split 256,
+    its fastest here)."""
     import attention_online_softmax_fwd_b200 as ab
     c = gen.CONFIGS["blasst_long_context"]
     B, Hq, Hkv, S, D = c["B"], c["Hq"], c["Hkv"], c["S"], c["D"]
     G = Hq // Hkv
     scale = gen.attn_scale(D)
     fl = prefill_flops(B, Hq, S, D)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
+    ws = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
     report = {"workload": "blasst_long_context B1 Hq32 Hkv8 S32768 D128, tiles of 64 keys",
-              "decode_note": "decode bytes = every K row + V rows of kept (KV head, tile) pairs; L2 flushed",
+              "decode_note": "decode bytes = every K row + V rows of kept (KV head, tile) pairs; L2 flushed; "
+                             "timed without the decision-mask output",
               "prefill_note": "prefill speedup against the dense kernel on the same input"}
     for name, amp, period, seed in (("recipe", 4.0, 64, c["seed"]), ("dominant_key", 12.0, S, c["seed"] + 7)):
         q_h, k_h, v_h = gen.peaked_prefill_inputs(B, Hq, Hkv, S, D, seed, amp=amp, period=period)
@@ -559,7 +601,8 @@ def blasst_long_context_report(dev, peaks, reps=5):
         ms0, (o0, _) = _timed(lambda: ab.prefill(q, k, v, causal=True, scale=scale), dev, 3)
         sec["prefill"]["0.0"] = {"ms": ms0, "tflops": fl / (ms0 * 1e-3) / 1e12}
         dense_bytes = decode_bytes([S], Hq, Hkv, D, cache.max_pages)
-        dms0, (do0, _) = _timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=256), dev, reps, flush)
+        dms0, (do0, _) = _timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=256, workspace=ws), dev,
+                                reps, flush)
         sec["decode"]["0.0"] = {"ms": dms0, "split": 256, "gbs": dense_bytes / (dms0 * 1e-3) / 1e9,
                                 "frac_of_measured_hbm": dense_bytes / (dms0 * 1e-3) / 1e9 / peaks["hbm_gbs"]}
         for lam in (0.1, 0.3):
@@ -573,49 +616,61 @@ def blasst_long_context_report(dev, peaks, reps=5):
                 "skipped_frac": float(((mask == 1) & vis).sum().item() / vis.sum().item()),
                 "max_abs_err_vs_dense": float(err.max().item()), "mean_abs_err_vs_dense": float(err.mean().item()),
                 "speedup_vs_dense": ms0 / ms}
-            for split in (2048, 256):
+            for split in (2048, 256, S):
                 for rows in ("group", "head"):
-                    ms, (do, _, dmask) = _timed(
-                        lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=split,
-                                                       rows_per_unit=rows), dev, reps, flush)
-                    dvis = dmask != 2
-                    k_b, v_kept = _decode_kept_bytes(dmask, [S], G, D, rows, c["page_size"], cache.max_pages)
-                    v_all = S * Hkv * D * 2
-                    kept_bytes = dense_bytes - v_all + v_kept      # q, o, lse and tables included
-                    sec["decode"][f"{lam}_split{split}_{rows}"] = {
-                        "ms": ms, "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
-                        "bytes_kept": kept_bytes, "v_bytes_saved_frac": 1.0 - v_kept / v_all,
-                        "gbs_on_kept_bytes": kept_bytes / (ms * 1e-3) / 1e9,
-                        "max_abs_err_vs_dense": float((do.float() - do0.float()).abs().max().item()),
-                        "speedup_vs_dense": dms0 / ms}
+                    sec["decode"][f"{lam}_split{split}_{rows}"] = _skip_decode_line(
+                        ab, dargs, lam, split, rows, [S], G, D, c["page_size"], cache.max_pages, dense_bytes, dms0,
+                        do0, scale, dev, reps, flush, ws)
         report[name] = sec
         del q, k, v, dargs
 
     # The same dominant-key pattern over a batch of 8 sequences of 16384 tokens (537 MB of K/V):
     # enough bytes that the decode is bound by HBM rather than by latency, so that the V rows the
-    # skip does not read show up in the time.
+    # skip does not read show up in the time. Split 16384 is one decision walk per sequence.
     cache = gen.peaked_decode_batch(8, Hq, Hkv, 16384, D, c["seed"] + 9, amp=12.0, page_size=c["page_size"])
     dargs = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
     lens = [16384] * 8
     dense_bytes = decode_bytes(lens, Hq, Hkv, D, cache.max_pages)
-    dms0, (do0, _) = _timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=256), dev, reps, flush)
+    dense = {sp: _timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=sp, workspace=ws), dev, reps,
+                        flush) for sp in (128, 256)}
+    best = min(dense, key=lambda sp: dense[sp][0])
+    dms0, (do0, _) = dense[best]
     batch = {"workload": "8 sequences x 16384 tokens, 12u on key 0 of each and on every query, Hq32 Hkv8 D128",
-             "0.0": {"ms": dms0, "split": 256, "gbs": dense_bytes / (dms0 * 1e-3) / 1e9}}
+             "0.0": {"ms": dms0, "split": best, "gbs": dense_bytes / (dms0 * 1e-3) / 1e9,
+                     "ms_by_split": {str(sp): dense[sp][0] for sp in dense}}}
     for lam in (0.1, 0.3):
-        for rows in ("group", "head"):
-            ms, (do, _, dmask) = _timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=2048,
-                                                                       rows_per_unit=rows), dev, reps, flush)
-            dvis = dmask != 2
-            k_b, v_kept = _decode_kept_bytes(dmask, lens, G, D, rows, c["page_size"], cache.max_pages)
-            v_all = sum(lens) * Hkv * D * 2
-            kept_bytes = dense_bytes - v_all + v_kept
-            batch[f"{lam}_split2048_{rows}"] = {
-                "ms": ms, "skipped_frac": float(((dmask == 1) & dvis).sum().item() / dvis.sum().item()),
-                "v_bytes_saved_frac": 1.0 - v_kept / v_all, "gbs_on_kept_bytes": kept_bytes / (ms * 1e-3) / 1e9,
-                "max_abs_err_vs_dense": float((do.float() - do0.float()).abs().max().item()),
-                "speedup_vs_dense": dms0 / ms}
+        for split in (256, 2048, 16384):
+            for rows in ("group", "head"):
+                batch[f"{lam}_split{split}_{rows}"] = _skip_decode_line(
+                    ab, dargs, lam, split, rows, lens, G, D, c["page_size"], cache.max_pages, dense_bytes, dms0,
+                    do0, scale, dev, reps, flush, ws)
     report["dominant_key_decode_batch"] = batch
     return report
+
+
+def skip_overhead_report(dev, reps=5):
+    """The tile-skip decode with nothing skipped (lambda = 1e-6 on the N(0, 1) batch of
+    64 sequences of 512..8192 tokens, split 256: one pass over K) against the dense
+    decode on the same batch: the cost of deciding every tile and gating its V rows."""
+    import attention_online_softmax_fwd_b200 as ab
+    dc = gen.CONFIGS["paged_gqa_decode"]
+    cache = gen.paged_decode_inputs(dc["N"], dc["Hq"], dc["Hkv"], dc["D"], dc["page_size"], dc["len_lo"],
+                                    dc["len_hi"], seed=dc["seed"], poison=False)
+    dargs = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+    scale = gen.attn_scale(dc["D"])
+    flush = L2Flush(dev)
+    ws = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    dms, _ = _timed(lambda: ab.decode_paged(*dargs, scale=scale, split_tokens=256, workspace=ws), dev, reps, flush)
+    out = {"workload": "paged_gqa_decode (64 sequences, 512..8192 tokens, Hq32 Hkv8 D128), split 256",
+           "dense_ms": dms}
+    for lam in (1e-6, 0.3):
+        cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+        ms, _ = _timed(lambda: ab.decode_paged_blasst(*dargs, lam, scale=scale, split_tokens=256, skip_mask=False,
+                                                      workspace=ws, skipped_tiles=cnt), dev, reps, flush)
+        out[str(lam)] = {"ms": ms, "time_vs_dense": ms / dms, "skipped_decisions": int(cnt.item()) // (reps + 1),
+                         "passes": ab.binding.decode_skip_passes(dc["N"], dc["Hq"], dc["Hkv"], cache.max_pages,
+                                                                 dc["page_size"], 256)}
+    return out
 
 
 def main():
