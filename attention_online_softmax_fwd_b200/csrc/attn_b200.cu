@@ -266,8 +266,8 @@ bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0
 // no chunk straddles a decision split), halved down to 64 while the batch gives fewer than 32768
 // (sequence, query head, chunk) triples, so that a few long sequences still fill the GPU.
 struct BlasstLayout {
-  int chunk = 0, max_chunks = 0, max_tiles = 0, tok64 = 0;
-  size_t o_off = 0, lse_off = 0, s_off = 0, tmax_off = 0, cmax_off = 0, total = 0;
+  int chunk = 0, max_chunks = 0, max_tiles = 0, tok64 = 0, chunk2 = 0, max_chunks2 = 0;
+  size_t o_off = 0, lse_off = 0, s_off = 0, tmax_off = 0, cmax_off = 0, cpre_off = 0, total = 0;
 };
 
 bool blasst_layout(int num_seqs, int Hq, int D, int max_pages, int page_size, int split_tokens, BlasstLayout* L) {
@@ -280,22 +280,25 @@ bool blasst_layout(int num_seqs, int Hq, int D, int max_pages, int page_size, in
   for (int c : {256, 192, 128}) {
     if (split_tokens % c == 0) { C = c; break; }
   }
+  L->chunk2 = C;   // pass 2's item
+  L->max_chunks2 = int((cap + C - 1) / C);
   while (C % 128 == 0 && (long long)num_seqs * Hq * ((cap + C - 1) / C) < 32768) C /= 2;
-  L->chunk = C;
+  L->chunk = C;    // pass 1's item
   L->max_chunks = int((cap + C - 1) / C);
   L->max_tiles = int((cap + 63) / 64);
   L->tok64 = L->max_tiles * 64;
   const size_t rows = size_t(num_seqs) * size_t(Hq);
-  size_t sz[5];
-  if (!mul_size(rows, size_t(L->max_chunks) * D * sizeof(float), &sz[0]) ||
-      !mul_size(rows, size_t(L->max_chunks) * sizeof(float), &sz[1]) ||
+  size_t sz[6];
+  if (!mul_size(rows, size_t(L->max_chunks2) * D * sizeof(float), &sz[0]) ||
+      !mul_size(rows, size_t(L->max_chunks2) * sizeof(float), &sz[1]) ||
       !mul_size(rows, size_t(L->tok64) * sizeof(float), &sz[2]) ||
       !mul_size(rows, size_t(L->max_tiles) * sizeof(float), &sz[3]) ||
-      !mul_size(rows, size_t(L->max_chunks) * sizeof(float), &sz[4]))
+      !mul_size(rows, size_t(L->max_chunks) * sizeof(float), &sz[4]) ||
+      !mul_size(rows, size_t(L->max_chunks) * sizeof(float), &sz[5]))
     return false;
   size_t off = kWsHeader;
-  size_t* offs[5] = {&L->o_off, &L->lse_off, &L->s_off, &L->tmax_off, &L->cmax_off};
-  for (int i = 0; i < 5; ++i) {
+  size_t* offs[6] = {&L->o_off, &L->lse_off, &L->s_off, &L->tmax_off, &L->cmax_off, &L->cpre_off};
+  for (int i = 0; i < 6; ++i) {
     *offs[i] = off;
     size_t end = 0;
     if (!add_size(off, sz[i], &end) || !add_size(end, 255, &end)) return false;
@@ -310,10 +313,10 @@ bool blasst_layout(int num_seqs, int Hq, int D, int max_pages, int page_size, in
 // while the split kernel's last CTAs run and waits (griddepcontrol.wait) for
 // that grid to finish and its writes to be visible before it reads the partials.
 // A row with more than 64 partials (long sequences at small splits) takes
-// sixteen warps on each of D / 32 CTAs, one per 32 head dimensions; four warps on
-// one CTA otherwise.
+// sixteen warps on each of D / 32 CTAs, one per 32 head dimensions (sixteen warps
+// on one CTA when the partials are sparse); four warps on one CTA otherwise.
 template <int D>
-int launch_merge(const DecodeParams& p, cudaStream_t stream) {
+int launch_merge(const DecodeParams& p, cudaStream_t stream, bool sparse = false) {
   const long long pairs = (long long)p.num_seqs * p.Hq;
   const bool wide = p.max_splits > 64;
   constexpr int kSlices = D / 32;
@@ -327,8 +330,15 @@ int launch_merge(const DecodeParams& p, cudaStream_t stream) {
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 16, kSlices>, p)
-                             : cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 4, 1>, p);
+  cudaError_t e;
+  if (wide && sparse) {   // few O rows to read: one CTA per row, its sixteen warps on the log-sum-exps
+    cfg.gridDim = dim3(unsigned(pairs));
+    e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 16, 1, true>, p);
+  } else if (wide)
+    e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 16, kSlices, false>, p);
+  else
+    e = sparse ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 4, 1, true>, p)
+               : cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 4, 1, false>, p);
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   return launch_status();
 }
@@ -405,8 +415,9 @@ int dispatch_decode_heads(int G, int hg, const CUtensorMap& tk, const CUtensorMa
   }
 }
 
-// Two-pass tile-skip decode: pass 1 (scores and maxima), pass 2 (decisions, kept V, P V) as a programmatic
-// dependent of pass 1, then the merge of the chunk partials as a programmatic dependent of pass 2.
+// Two-pass tile-skip decode: pass 1 (scores and maxima); for splits of more than 16 chunks the scan of the
+// running maxima at the chunk starts; pass 2 (decisions, kept V, P V); the merge of the chunk partials (reading
+// only the non-empty ones when lambda > 0) -- each a programmatic dependent of the one before.
 template <int D, int G, int HG, bool PER_HEAD>
 int launch_blasst(const CUtensorMap& tk, const CUtensorMap& tvg, const CUtensorMap& tvh, const DecodeParams& p,
                   int* tickets, int sms, cudaStream_t stream) {
@@ -415,6 +426,7 @@ int launch_blasst(const CUtensorMap& tk, const CUtensorMap& tvg, const CUtensorM
   if (int st = set_smem_once<decode_scores_kernel<D, G, HG>>(L1::kDynamic)) return st;
   if (int st = set_smem_once<decode_pv_kernel<D, G, HG, PER_HEAD>>(L2::kDynamic)) return st;
   const long long items = (long long)p.max_chunks * p.num_seqs * (p.Hkv / HG);
+  const long long items2 = (long long)p.max_chunks2 * p.num_seqs * (p.Hkv / HG);
   const long long slots1 = (long long)sms * L1::kBlocks, slots2 = (long long)sms * L2::kBlocks;
   decode_scores_kernel<D, G, HG><<<dim3(unsigned(items < slots1 ? items : slots1)), dim3((HG + 1) * 32),
                                    L1::kDynamic, stream>>>(tk, p, tickets);
@@ -423,7 +435,18 @@ int launch_blasst(const CUtensorMap& tk, const CUtensorMap& tvg, const CUtensorM
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(items < slots2 ? items : slots2));
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (p.ws_cpre) {   // long splits: running maxima at the chunk starts, between the passes
+    const long long rows = (long long)p.num_seqs * p.Hq;
+    cfg.gridDim = dim3(unsigned((rows + kScanWarps - 1) / kScanWarps));
+    cfg.blockDim = dim3(kScanWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&cfg, decode_chunk_prefix_kernel, p) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (int st = launch_status()) return st;
+  }
+  cfg.gridDim = dim3(unsigned(items2 < slots2 ? items2 : slots2));
   cfg.blockDim = dim3((HG + 1) * 32);
   cfg.dynamicSmemBytes = L2::kDynamic;
   cfg.stream = stream;
@@ -432,10 +455,10 @@ int launch_blasst(const CUtensorMap& tk, const CUtensorMap& tvg, const CUtensorM
   if (cudaLaunchKernelEx(&cfg, decode_pv_kernel<D, G, HG, PER_HEAD>, tvg, tvh, p, tickets + 1) != cudaSuccess)
     return ATTN_ERR_CUDA;
   if (int st = launch_status()) return st;
-  DecodeParams pm = p;          // the merge combines chunk partials
-  pm.split_tokens = p.chunk_tokens;
-  pm.max_splits = p.max_chunks;
-  return launch_merge<D>(pm, stream);
+  DecodeParams pm = p;          // the merge combines the pass-2 item partials
+  pm.split_tokens = p.chunk2_tokens;
+  pm.max_splits = p.max_chunks2;
+  return launch_merge<D>(pm, stream, p.log2_lambda != -INFINITY);
 }
 
 template <int D, int HG, bool PER_HEAD>
@@ -739,8 +762,12 @@ static int decode_impl(const void* q, const void* k_pages, const void* v_pages, 
     p.ws_s = reinterpret_cast<float*>(ws + BL.s_off);
     p.ws_tmax = reinterpret_cast<float*>(ws + BL.tmax_off);
     p.ws_cmax = reinterpret_cast<float*>(ws + BL.cmax_off);
+    // splits of more than 16 chunks: the running maximum at each chunk start is scanned between the passes
+    p.ws_cpre = split_tokens / BL.chunk > 16 ? reinterpret_cast<float*>(ws + BL.cpre_off) : nullptr;
     p.chunk_tokens = BL.chunk;
     p.max_chunks = BL.max_chunks;
+    p.chunk2_tokens = BL.chunk2;
+    p.max_chunks2 = BL.max_chunks2;
     p.tok64 = BL.tok64;
     const uint32_t gbox[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), uint32_t(bhg), 1};
     const uint32_t box1[5] = {64, uint32_t(kDhChunk), uint32_t(D / 64), 1, 1};

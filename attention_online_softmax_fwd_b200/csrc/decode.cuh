@@ -54,8 +54,11 @@ struct DecodeParams {
   float* ws_s;        // scaled scores (log2 units) [N][Hkv / HG][tok64][HG][G]
   float* ws_tmax;     // row maxima of every 64-token tile [N][Hq][max_tiles]
   float* ws_cmax;     // row maxima of every chunk [N][Hq][max_chunks]
+  float* ws_cpre;     // splits of more than 16 chunks: running maximum at every chunk start [N][Hq][max_chunks],
+                      // else null
   unsigned long long* skipped_tiles;   // count of skipped decisions, or null
-  int chunk_tokens, max_chunks, tok64;
+  int chunk_tokens, max_chunks, tok64;   // pass 1's work item (chunk maxima per chunk)
+  int chunk2_tokens, max_chunks2;        // pass 2's work item (a multiple of chunk_tokens, one partial each)
 };
 
 constexpr int kDecTile = 64;          // tokens per tile (= BLASST decision tile)
@@ -596,9 +599,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // running maximum; the W warps then combine in a fixed order (deterministic).
 // W = 4 serves batches of many sequences; W = 16 with one slice per 32 head
 // dimensions puts many partials in flight on many SMs for the few rows of a
-// long single sequence.
+// long single sequence. SPARSE (the tile-skip decode's chunk partials, most of
+// them empty when most tiles are skipped) reads a partial's O row only when
+// its log-sum-exp is finite.
 constexpr int kMergeChunk = 8;   // splits per warp in flight
-template <int D, int W = 4, int DS = 1>
+template <int D, int W = 4, int DS = 1, bool SPARSE = false>
 __global__ void __launch_bounds__(W * 32) decode_merge_kernel(const DecodeParams p) {
   static_assert((D / 32) % DS == 0, "a slice gives each lane whole floats");
   constexpr int kMergeWarps = W;
@@ -635,14 +640,21 @@ __global__ void __launch_bounds__(W * 32) decode_merge_kernel(const DecodeParams
   float m = neg_inf, wsum = 0.f;
   for (int base = warp; base < n_splits; base += kMergeWarps * kMergeChunk) {
     float ls[kMergeChunk], ov[kMergeChunk][DL];
+    if constexpr (SPARSE) {   // most partials empty (skipped chunks): their O rows are not read
+#pragma unroll
+      for (int u = 0; u < kMergeChunk; ++u) {
+        const int su = base + u * kMergeWarps;
+        ls[u] = su < n_splits ? lse_base[size_t(su) * p.Hq] : neg_inf;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < kMergeChunk; ++u) {
       const int su = base + u * kMergeWarps;
-      ls[u] = neg_inf;
+      if constexpr (!SPARSE) ls[u] = neg_inf;
 #pragma unroll
       for (int d = 0; d < DL; ++d) ov[u][d] = 0.f;
-      if (su < n_splits) {
-        ls[u] = lse_base[size_t(su) * p.Hq];
+      if (SPARSE ? ls[u] != neg_inf : su < n_splits) {
+        if constexpr (!SPARSE) ls[u] = lse_base[size_t(su) * p.Hq];
         const float* src = o_base + size_t(su) * o_stride;
         if constexpr (DL == 4) {
           const float4 t = *reinterpret_cast<const float4*>(src);

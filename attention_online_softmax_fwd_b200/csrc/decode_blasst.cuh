@@ -296,6 +296,64 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
   __syncthreads();
 }
 
+// ---------------------------------------------------------------- between the passes (long splits)
+
+// The exclusive running maximum of the chunk maxima within each decision split:
+// ws_cpre[row][ch] = maximum of ws_cmax[row][j] over the chunks j < ch of ch's split,
+// -inf for a split's first chunk. One warp per (sequence, query head) row: a segmented
+// max-scan over 32 chunks at a time (segments = splits), carried from block to block,
+// with kScanBatch blocks loaded before they are scanned.
+constexpr int kScanWarps = 4;
+constexpr int kScanBatch = 8;
+__global__ void __launch_bounds__(kScanWarps * 32) decode_chunk_prefix_kernel(const DecodeParams p) {
+  launch_dependents();     // pass 2 may be scheduled early; it waits for this grid
+  grid_dependency_wait();  // pass 1's chunk maxima
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kScanWarps + warp;   // seq * Hq + hq
+  if (row >= (long long)p.num_seqs * p.Hq) return;
+  const float neg_inf = -__int_as_float(0x7f800000);
+  const int seq = int(row / p.Hq);
+  const int capacity = p.max_pages * p.page_size;
+  int len = __ldg(&p.seq_lens[seq]);
+  len = len < 0 ? 0 : min(len, capacity);
+  const int C = p.chunk_tokens;
+  const int nch = (len + C - 1) / C;
+  const int cps = p.split_tokens / C;   // chunks per split
+  const float* cm = p.ws_cmax + size_t(row) * p.max_chunks;
+  float* cp = p.ws_cpre + size_t(row) * p.max_chunks;
+  float carry = neg_inf;
+  for (int base = 0; base < nch; base += 32 * kScanBatch) {
+    float v[kScanBatch];
+#pragma unroll
+    for (int b = 0; b < kScanBatch; ++b) {
+      const int ch = base + b * 32 + lane;
+      v[b] = ch < nch ? cm[ch] : neg_inf;
+    }
+#pragma unroll
+    for (int b = 0; b < kScanBatch; ++b) {
+      if (base + b * 32 >= nch) break;
+      const int ch = base + b * 32 + lane;
+      const bool start = ch % cps == 0;
+      // inclusive scan: (value, "a split starts in my window") combined with the window to the left
+      float inc = v[b];
+      int fl = start ? 1 : 0;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const float ov = __shfl_up_sync(0xffffffffu, inc, d);
+        const int of = __shfl_up_sync(0xffffffffu, fl, d);
+        if (lane >= d) {
+          if (!fl) inc = fmaxf(inc, ov);
+          fl |= of;
+        }
+      }
+      if (!fl) inc = fmaxf(inc, carry);   // no split start between the block's start and this chunk
+      const float left = __shfl_up_sync(0xffffffffu, inc, 1);
+      if (ch < nch) cp[ch] = start ? neg_inf : (lane == 0 ? carry : left);
+      carry = __shfl_sync(0xffffffffu, inc, 31);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- pass 2
 
 // What the pass-2 producer tells the consumers about a stage.
@@ -353,8 +411,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
   const int lane = threadIdx.x & 31;
   const int capacity = p.max_pages * p.page_size;
   const int n_groups = p.Hkv / HG;
-  const int C = p.chunk_tokens;
-  const long long num_items = (long long)p.max_chunks * p.num_seqs * n_groups;
+  const int C = p.chunk_tokens;     // pass-1 chunk (the granularity of the chunk maxima)
+  const int C2 = p.chunk2_tokens;   // this pass's work item, a whole number of pass-1 chunks
+  const long long num_items = (long long)p.max_chunks2 * p.num_seqs * n_groups;
   const float neg_inf = -__int_as_float(0x7f800000);
 
   if (threadIdx.x == 0) {
@@ -395,17 +454,24 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
         int sq, ch, gr;
         dh_item_coords(t, p.num_seqs, n_groups, sq, ch, gr);
         nx_len = __ldg(&p.seq_lens[sq]);
-        const int e = (((ch * C) / p.page_size) & ~31) + lane;
+        const int e = (((ch * C2) / p.page_size) & ~31) + lane;
         nx_win = e < p.max_pages ? __ldg(&p.block_table[size_t(sq) * p.max_pages + e]) : -1;
         const size_t rb = size_t(sq) * p.Hq + (lane < R ? gr * R + lane : 0);
-        const int ta = ch * C / kDecTile;
+        const int ta = ch * C2 / kDecTile;
+        const int c1 = ch * C2 / C;   // the item's first pass-1 chunk
 #pragma unroll
         for (int i = 0; i < kBlChunkTiles; ++i)   // tiles past the sequence end are read, never used
           nx_tm[i] = (lane < R && ta + i < p.max_tiles) ? p.ws_tmax[rb * p.max_tiles + ta + i] : neg_inf;
-        const int j0 = (ch * C / p.split_tokens) * (p.split_tokens / C);
+        if (p.ws_cpre) {   // long splits: the running maximum at the chunk start, computed between the passes
+          nx_cm[0] = lane < R ? p.ws_cpre[rb * p.max_chunks + c1] : neg_inf;
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          nx_cm[u] = (lane < R && j0 + u < ch) ? p.ws_cmax[rb * p.max_chunks + j0 + u] : neg_inf;
+          for (int u = 1; u < 16; ++u) nx_cm[u] = neg_inf;
+        } else {
+          const int j0 = (ch * C2 / p.split_tokens) * (p.split_tokens / C);
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            nx_cm[u] = (lane < R && j0 + u < c1) ? p.ws_cmax[rb * p.max_chunks + j0 + u] : neg_inf;
+        }
       }
     };
     fetch_next();
@@ -424,9 +490,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
       int seq, chunk, grp;
       dh_item_coords(item, p.num_seqs, n_groups, seq, chunk, grp);
       if (len > capacity || len < 0) len = len < 0 ? 0 : capacity;   // reported by pass 1
-      const int t_begin = chunk * C;
+      const int t_begin = chunk * C2;
       if (t_begin >= len) continue;
-      const int t_end = min(t_begin + C, len);
+      const int t_end = min(t_begin + C2, len);
 
       // ---- decisions of the chunk's tiles
       const int hq = grp * R + lane;
@@ -435,14 +501,16 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
 #pragma unroll
       for (int i = 0; i < kBlChunkTiles; ++i)
         if (i >= nt) tm[i] = neg_inf;
-      {
-        // chunk maxima beyond the first sixteen of the split (splits longer than 16 chunks)
+      if (!p.ws_cpre) {
+        // chunk maxima beyond the first sixteen of the split (splits of 17 to 32 chunks; longer ones
+        // have the running maximum at each chunk start computed between the passes)
         const int j0 = (t_begin / p.split_tokens) * (p.split_tokens / C) + 16;
         const float* cm = p.ws_cmax + row_base * p.max_chunks;
-        for (int jb = j0; jb < chunk; jb += 16) {
+        const int c1 = t_begin / C;
+        for (int jb = j0; jb < c1; jb += 16) {
           float v[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) v[u] = (lane < R && jb + u < chunk) ? cm[jb + u] : neg_inf;
+          for (int u = 0; u < 16; ++u) v[u] = (lane < R && jb + u < c1) ? cm[jb + u] : neg_inf;
 #pragma unroll
           for (int u = 0; u < 16; ++u) m = fmaxf(m, v[u]);
         }
@@ -482,6 +550,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
         n_skipped += __popc(__ballot_sync(0xffffffffu, unit_lane && !kept));
       }
       if (p.skipped_tiles && lane == 0 && n_skipped) atomicAdd(p.skipped_tiles, (unsigned long long)n_skipped);
+      if (last_kept < 0 && len > C2) {
+        // nothing kept (only with lambda > 0): the chunk's partial is empty, and the merge reads no O
+        // row whose log-sum-exp is -inf -- written here, with no stage for the consumers
+        if (lane < R) p.ws_lse[(size_t(seq) * p.max_chunks2 + chunk) * p.Hq + hq] = neg_inf;
+        continue;
+      }
 
       // ---- stream the stages of the kept tiles (one empty stage if the chunk keeps nothing)
       const int32_t* bt_row = p.block_table + size_t(seq) * p.max_pages;
@@ -645,7 +719,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
         lr_part[c] += __shfl_xor_sync(0xffffffffu, lr_part[c], 8);
         lr_part[c] += __shfl_xor_sync(0xffffffffu, lr_part[c], 16);
       }
-      const int n_chunks = (len + C - 1) / C;
+      const int n_chunks = (len + C2 - 1) / C2;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         if (!head_valid[c]) continue;
@@ -663,14 +737,17 @@ __global__ void __launch_bounds__((HG + 1) * 32, 3)
             p.lse[size_t(seq) * p.Hq + hq] = lsum > 0.f ? (mr[c] + __log2f(lsum)) * 0.69314718055994531f : neg_inf;
         } else {
           const uint64_t keep = l2_keep_policy();
-          float* dst = p.ws_o + ((size_t(seq) * p.max_chunks + chunk) * p.Hq + hq) * D + g;
+          float* dst = p.ws_o + ((size_t(seq) * p.max_chunks2 + chunk) * p.Hq + hq) * D + g;
+          // with lambda > 0 the merge reads an O row only when its log-sum-exp is finite
+          if (lsum > 0.f || p.log2_lambda == neg_inf) {
 #pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            st_keep(dst + 16 * m, o[m][c] * inv, keep);
-            st_keep(dst + 16 * m + 8, o[m][c + 2] * inv, keep);
+            for (int m = 0; m < MT; ++m) {
+              st_keep(dst + 16 * m, o[m][c] * inv, keep);
+              st_keep(dst + 16 * m + 8, o[m][c + 2] * inv, keep);
+            }
           }
           if (g == 0)
-            st_keep(&p.ws_lse[(size_t(seq) * p.max_chunks + chunk) * p.Hq + hq],
+            st_keep(&p.ws_lse[(size_t(seq) * p.max_chunks2 + chunk) * p.Hq + hq],
                     lsum > 0.f ? mr[c] + __log2f(lsum) : neg_inf, keep);
         }
       }

@@ -673,6 +673,55 @@ def skip_overhead_report(dev, reps=5):
     return out
 
 
+PROFILE_CASES = ("skip_decode_one_pass", "skip_decode_two_pass", "dense_decode_batch", "single_seq_decode",
+                 "mha_prefill")
+
+
+def run_profile_case(name, dev, calls=5):
+    """A few launches of one workload, for an ncu capture of its kernels (nothing is timed or
+    printed but a line naming the case):
+      skip_decode_one_pass  the paged GQA decode batch (64 sequences of 512..8192 tokens),
+                            lambda = 0.3, split 256, group decisions: one pass over K
+      skip_decode_two_pass  8 x 16384 tokens with one dominant key each, lambda = 0.3, one
+                            split per sequence, group decisions: two passes
+      dense_decode_batch    the same 8 x 16384 tokens, dense, split 256
+      single_seq_decode     the 32768-token BLASST sequence's last row, dense, split 256
+      mha_prefill           the MHA prefill B4 Hq=Hkv=32 S2048 D128, causal"""
+    import attention_online_softmax_fwd_b200 as ab
+    scale = gen.attn_scale(128)
+    ws = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    if name == "mha_prefill":
+        c = gen.CONFIGS["mha_prefill_llama2_7b"]
+        q, k, v = [t.to(dev) for t in gen.prefill_inputs(c["B"], c["Hq"], c["Hkv"], c["S"], c["D"], c["seed"])]
+        fn = lambda: ab.prefill(q, k, v, causal=True, scale=scale)
+    else:
+        if name == "skip_decode_one_pass":
+            dc = gen.CONFIGS["paged_gqa_decode"]
+            cache = gen.paged_decode_inputs(dc["N"], dc["Hq"], dc["Hkv"], dc["D"], dc["page_size"], dc["len_lo"],
+                                            dc["len_hi"], seed=dc["seed"], poison=False)
+        elif name == "single_seq_decode":
+            c = gen.CONFIGS["blasst_long_context"]
+            q_h, k_h, v_h = gen.peaked_prefill_inputs(1, c["Hq"], c["Hkv"], c["S"], c["D"], c["seed"] + 7, amp=12.0,
+                                                      period=c["S"])
+            cache = gen.paged_from_contiguous(q_h[:, -1], k_h, v_h, page_size=c["page_size"], seed=c["seed"] + 1,
+                                              poison=False)
+        else:
+            cache = gen.peaked_decode_batch(8, 32, 8, 16384, 128, gen.CONFIGS["blasst_long_context"]["seed"] + 9,
+                                            amp=12.0, page_size=16)
+        d = [t.to(dev) for t in (cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens)]
+        if name == "skip_decode_one_pass":
+            fn = lambda: ab.decode_paged_blasst(*d, 0.3, scale=scale, split_tokens=256, skip_mask=False, workspace=ws)
+        elif name == "skip_decode_two_pass":
+            fn = lambda: ab.decode_paged_blasst(*d, 0.3, scale=scale, split_tokens=16384, skip_mask=False,
+                                                workspace=ws)
+        else:
+            fn = lambda: ab.decode_paged(*d, scale=scale, split_tokens=256, workspace=ws)
+    for _ in range(calls):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "calls": calls}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -683,7 +732,12 @@ def main():
     ap.add_argument("--no-blasst", action="store_true", help="skip the long-context BLASST report")
     ap.add_argument("--no-extras", action="store_true", help="skip the FP8-decode and chunked-prefill reports")
     ap.add_argument("--cpu-heads", type=int, default=8)
+    ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
+                    help="run a few launches of one workload for an ncu capture, and nothing else")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case, torch.device("cuda:0"))
+        return
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup(args.gpus)

@@ -175,7 +175,7 @@ int attn_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_
  * The decode splits each sequence's keys into chunks of split_tokens tokens,
  * computes one partial (O, LSE) per (sequence, query head, chunk), and merges
  * them. The workspace holds a 256-byte header (the kernel's work counter,
- * reset by the library on every call) and those partials:
+ * reset by the library on every call that uses it) and those partials:
  *   fp32 [num_seqs][max_splits][Hq][D] (padded to 256 B) + fp32 [num_seqs][max_splits][Hq]
  * with max_splits = ceil(max_pages_per_seq * page_size / split_tokens).
  * Returns 0 for invalid arguments or a size that does not fit a size_t.
@@ -192,12 +192,16 @@ size_t attn_decode_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_pe
  * walked in token order and a tile's V rows are read after its decision. Two
  * passes, for batches with too few splits to fill the GPU: the first computes
  * the scaled scores of every cached token and query head, and the row maxima
- * of every 64-token tile and of every work chunk; the second derives the
- * decisions from the maxima and reads V only for kept tiles. The size covers
- * both: the scores (fp32 [num_seqs][Hq][padded tokens]), the maxima, and one
- * partial (O, LSE) per (sequence, query head, chunk); a chunk is at most 256
- * tokens and divides split_tokens. Returns 0 for invalid arguments or an
- * overflowing size.
+ * of every 64-token tile and of every chunk of its work; the second derives
+ * the decisions from the maxima and reads V only for kept tiles. The second
+ * pass's item is the largest of 256, 192, 128 and 64 tokens that divides
+ * split_tokens; the first pass's chunk is that item, halved down to 64 tokens
+ * while the batch has fewer than 32768 (sequence, query head, chunk) triples.
+ * The size covers both paths: the scores (fp32 [num_seqs][Hq][padded
+ * tokens]), the tile and chunk maxima, the running maximum at every chunk
+ * start (used for splits of more than 16 chunks), and one partial (O, LSE)
+ * per (sequence, query head, second-pass item). Returns 0 for invalid
+ * arguments or an overflowing size.
  */
 size_t attn_decode_blasst_workspace_bytes(int num_seqs, int Hq, int D, int max_pages_per_seq,
                                           int page_size, int split_tokens);

@@ -105,12 +105,13 @@ def _blasst_layout(n, hq, d, mp, ps, sp):
     """The tile-skip workspace as the header documents it (chunk choice included)."""
     cap = mp * ps
     c = next((x for x in (256, 192, 128) if sp % x == 0), 64)
+    items2 = -(-cap // c)   # the second pass's items (one partial each)
     while c % 128 == 0 and n * hq * -(-cap // c) < 32768:
         c //= 2
     chunks, tiles = -(-cap // c), -(-cap // 64)
     r256 = lambda x: -(-x // 256) * 256
-    parts = [n * hq * chunks * d * 4, n * hq * chunks * 4, n * hq * tiles * 64 * 4, n * hq * tiles * 4,
-             n * hq * chunks * 4]
+    parts = [n * hq * items2 * d * 4, n * hq * items2 * 4, n * hq * tiles * 64 * 4, n * hq * tiles * 4,
+             n * hq * chunks * 4, n * hq * chunks * 4]
     return 256 + sum(r256(x) for x in parts), c
 
 
