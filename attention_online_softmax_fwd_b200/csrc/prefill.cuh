@@ -58,6 +58,9 @@ constexpr int kPfKeys = 128;     // keys per K/V tile (two 64-key decision tiles
 constexpr int kPfThreads = 384;
 constexpr int kPfProducerWarp = 0, kPfIssuerWarp0 = 1;   // issuer of tile x: warp 1 + x
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Chunked (paged) prefill: up to this many (sequence, query block) pairs are ranked by their
+// number of K/V tiles at the start of every CTA, so that the items go out longest first.
+constexpr int kPfMaxPairs = 256;
 // setmaxnreg split: warps 0-3 drop to kPfRegsLow registers, the softmax warps rise to
 // kPfRegsHigh. Per sub-partition: low + 2 * high <= 3 * 168, the launch allocation.
 constexpr int kPfRegsLow = 72, kPfRegsHigh = 216;
@@ -80,9 +83,11 @@ struct PrefillSmem {
                        bTeardown = 14, bKVFull = 15, bKVEmpty = 15 + kStages, kNumBars = 15 + 2 * kStages;
   static constexpr int kMisc = kBars + 8 * kNumBars;            // tmem base, flags
   static constexpr int kVotes = (kMisc + 16 + 15) / 16 * 16;    // skip votes [2][4][4] ints
-  static constexpr int kTotal = kMisc + 256;
-  static_assert(kVotes + 128 <= kTotal, "skip votes exceed the misc area");
+  static constexpr int kOrder = kMisc + 256;                    // paged: item costs and their order (below)
+  static constexpr int kTotal = kOrder + kPfMaxPairs * 6;
+  static_assert(kVotes + 128 <= kOrder, "skip votes exceed the misc area");
   static constexpr int kDynamic = kTotal + 1024;
+  static_assert(kDynamic <= 232448, "shared memory per block");
 };
 
 // TMEM columns: S_A | S_B | O_A | O_B
@@ -408,17 +413,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   // The CTA's items: round r takes item r * grid + b, with the CTA order b
   // reversed on odd rounds (a snake), so that the CTAs that take the longer
   // item of one round take the shorter of the next: with items in decreasing
-  // causal length, every CTA ends within about one tile of the others. The
-  // chunked (paged) prefill keeps the plain stride: there an item's length also
-  // depends on its sequence's cached prefix, the order is not monotonic, and
-  // the snake pairs long items with long ones (measured 15 % slower).
+  // length, every CTA ends within about one tile of the others. In the chunked
+  // (paged) prefill an item's length also depends on its sequence's cached
+  // prefix, so its items are put in that order first (ranked below); beyond
+  // kPfMaxPairs pairs they keep the (query block, sequence) order and the plain
+  // stride, since the snake over an unsorted order pairs long items with long
+  // ones (measured 15 % slower).
+  // The chunked (paged) prefill ranks its (sequence, query block) pairs by their K/V tile
+  // count, in shared memory, so that its items also go out longest first (pf_rank_pairs below).
+  const int n_pairs = p.B * p.n_qblocks;
+  const bool ranked = PAGED && n_pairs <= kPfMaxPairs;
+  const uint16_t* pair_order = reinterpret_cast<const uint16_t*>(smem + L::kOrder + kPfMaxPairs * 4);
   auto pf_item_of = [&](int round) {
-    const int b = (!PAGED && (round & 1)) ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x);
+    const int b = ((!PAGED || ranked) && (round & 1)) ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x);
     return round * int(gridDim.x) + b;
   };
   // Item decode shared by all roles: longest causal blocks first; the G query
   // heads of one KV head are adjacent so their K/V tiles are reused from L2.
   auto item_coords = [&](int item, int& qb, int& b, int& hq) {
+    if (ranked) {
+      const int pair = pair_order[item / p.Hq];
+      b = pair / p.n_qblocks;
+      qb = pair % p.n_qblocks;
+      hq = item % p.Hq;
+      return;
+    }
     const int per = p.B * p.Hq;
     qb = p.n_qblocks - 1 - item / per;
     const int rem = item % per;
@@ -447,6 +466,30 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (CAUSAL) return (off + qb * 2 * kPfRows + x * kPfRows + rows - 1) / kPfKeys + 1;
     return (p.S + kPfKeys - 1) / kPfKeys;
   };
+
+  if (ranked) {
+    // Rank the pairs by K/V tiles (both query tiles' counts), most first, ties in pair order:
+    // with the items in that order the snake gives every CTA about the same work, whatever the
+    // sequences' cached prefixes. Every CTA computes the same order.
+    uint32_t* cost = reinterpret_cast<uint32_t*>(smem + L::kOrder);
+    uint16_t* order = reinterpret_cast<uint16_t*>(smem + L::kOrder + kPfMaxPairs * 4);
+    for (int i = int(threadIdx.x); i < n_pairs; i += int(blockDim.x)) {
+      const int b = i / p.n_qblocks, qb = i % p.n_qblocks;
+      const int off = seq_offset(b, false);
+      cost[i] = uint32_t(tile_nkv(qb, 0, tile_rows(qb, 0), off) + tile_nkv(qb, 1, tile_rows(qb, 1), off));
+    }
+    __syncthreads();
+    for (int i = int(threadIdx.x); i < n_pairs; i += int(blockDim.x)) {
+      const uint32_t c = cost[i];
+      int rank = 0;
+      for (int j = 0; j < n_pairs; ++j) {
+        const uint32_t cj = cost[j];
+        rank += (cj > c || (cj == c && j < i)) ? 1 : 0;
+      }
+      order[rank] = uint16_t(i);
+    }
+    __syncthreads();
+  }
 
   // Register split: warps 0-3 give up registers, the softmax warpgroups take them
   // (kPfRegPoolNeeded is checked against the launch allocation on the host).
