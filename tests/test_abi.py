@@ -255,3 +255,16 @@ def test_decode_fp8_valid_arguments_without_a_device_report_cuda_error(lib):
     if torch.cuda.is_available():
         pytest.skip("a device is present")
     assert _decode_fp8(lib) == CUDA
+
+
+@pytest.mark.parametrize("args,want", [((64, 32, 8, 512, 16, 256), 1),      # 64 x 8 x 32 splits = 16384 triples
+                                       ((8, 32, 8, 1024, 16, 2048), 2),     # 8 x 8 x 8 = 512
+                                       ((8, 32, 8, 4096, 16, 2048), 1),     # 8 x 8 x 32 = 2048
+                                       ((1, 32, 8, 2048, 16, 256), 2),      # one 32K sequence: 1024
+                                       ((4, 64, 4, 64, 16, 64), 1),         # Hq / Hkv = 16: one pass always
+                                       ((0, 32, 8, 64, 16, 64), 0), ((4, 24, 8, 64, 16, 64), 0),
+                                       ((4, 32, 8, 64, 24, 64), 0), ((4, 32, 8, 64, 16, 96), 0),
+                                       ((4, 96, 3, 64, 16, 64), 0)])        # Hq / Hkv = 32
+def test_decode_skip_passes(lib, args, want):
+    assert lib.attn_decode_skip_passes(*args) == want
+    assert ab.binding.decode_skip_passes(*args) == want

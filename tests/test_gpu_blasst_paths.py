@@ -172,3 +172,44 @@ def test_decode_blasst_dominant_key_batch(cuda_device, split, passes):
                                                                       c.seq_lens, 16, scale, m, rows_per_unit=rows),
                             label=f"dominant batch {rows} split {split}")
         assert st["skipped"] > 0 and counted == st["skipped_gpu"]
+
+
+@pytest.mark.parametrize("passes", [1, 2])
+@pytest.mark.parametrize("rows", ["group", "head"])
+def test_decode_blasst_bad_page_raises_device_status(cuda_device, passes, rows):
+    """Out-of-range block-table entries on either skip path are never dereferenced:
+    the caller's status word reads ATTN_ERR_DEVICE_BOUNDS and the sequences whose
+    tables are valid match the oracle."""
+    lens = [300, 700, 1300, 2049]
+    split = 256
+    mp = -(-max(lens) // 16)
+    if passes == 1:
+        mp = max(mp, -(-ONE_PASS_MIN // (len(lens) * 2)) * split // 16)
+    c = _cache(8, 2, 128, 16, seed=5500, lens=lens, max_pages=mp)
+    c.block_table[1, 3] = c.num_pages + 5
+    c.block_table[2, 0] = -7
+    assert _passes(c, split) == passes
+    args = [t.to(cuda_device) for t in (c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens)]
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    scale = gen.attn_scale(128)
+    o, lse, mask = ab.decode_paged_blasst(*args, 0.5, scale=scale, split_tokens=split, rows_per_unit=rows,
+                                          device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 4                        # ATTN_ERR_DEVICE_BOUNDS
+    good = [0, 3]
+    o_ref, lse_ref, m_ref, margin = orc.decode_paged_blasst(c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens,
+                                                            16, scale, 0.5, split, rows_per_unit=rows, seqs=good)
+    m_ref = m_ref[good]
+    st = compare_blasst(o, lse, mask[good], o_ref, lse_ref, m_ref, margin[good],
+                        lambda m: orc.decode_paged_with_skip_mask(c.q, c.k_pages, c.v_pages, c.block_table,
+                                                                  c.seq_lens, 16, scale, _full_mask(m, mask, good),
+                                                                  rows_per_unit=rows, seqs=good),
+                        label=f"bad pages, {passes} pass, {rows}", select=lambda oo, ll: (oo[good], ll[good]))
+    assert st["decisions"] > 0
+
+
+def _full_mask(m_good, mask_gpu, good):
+    """The GPU's mask with the rows of the checked sequences replaced by ``m_good``."""
+    full = mask_gpu.cpu().numpy().copy()
+    full[good] = m_good
+    return full
