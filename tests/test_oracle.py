@@ -676,3 +676,30 @@ def test_decode_with_skip_mask_matches_brute_force():
     od, ld = orc.decode_paged(cache.q, cache.k_pages, cache.v_pages, cache.block_table, cache.seq_lens, 16, scale)
     np.testing.assert_allclose(o, od, atol=1e-12)
     np.testing.assert_allclose(lse, ld, atol=1e-12)
+
+
+def test_oracle_reproduces_its_golden_fixtures():
+    """tests/golden/oracle_fixtures.json holds the oracle's answers for two small
+    seeded cases (written by tests/golden/make_fixtures.py): recomputing them must
+    give the same values, so any change to the oracle's arithmetic is visible."""
+    import importlib.util
+    import json
+    import os
+    here = os.path.join(os.path.dirname(__file__), "golden")
+    spec = importlib.util.spec_from_file_location("make_fixtures", os.path.join(here, "make_fixtures.py"))
+    mf = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mf)
+    stored = json.load(open(os.path.join(here, "oracle_fixtures.json")))
+    fresh = mf.build()
+    for case in ("tiny_gqa_prefill", "blasst_paged_decode"):
+        for key, val in stored[case].items():
+            got = fresh[case][key]
+            if isinstance(val, list) and val and isinstance(val[0], (float, int, str)):
+                a = np.array([float(x) for x in val])
+                b = np.array([float(x) for x in got])
+                assert a.shape == b.shape, (case, key)
+                fin = np.isfinite(a)
+                assert np.array_equal(fin, np.isfinite(b)) and np.array_equal(a[~fin], b[~fin]), (case, key)
+                assert np.allclose(a[fin], b[fin], rtol=2e-7, atol=1e-12), (case, key)
+            else:
+                assert val == got, (case, key)
