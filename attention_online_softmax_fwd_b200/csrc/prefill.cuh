@@ -622,8 +622,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 if (tile == 0) {
                   prev_dropped = false;   // a unit's first tile is never dropped
                 } else if (pend_tag0 | pend_tag1) {
-                  // the previous tile's votes (loaded at once): in by now, since Q K^T of this tile,
-                  // issued after they were cast, has completed
+                  // the previous tile's votes (loaded at once): cast right after its scores were read,
+                  // normally in by the time the ring has a slot for this V tile
                   const int d = pf_dropped_by_both(votes, pend_tag0, pend_tag1, abort_flag, p.status, wait_lim);
                   if (d < 0) { ok = false; break; }
                   prev_dropped = d == 3;
@@ -808,12 +808,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int key0 = j * kPfKeys;
         float s[kPfKeys];
         pf_load_scores<CAUSAL>(taddr_s, s, key0, off + row, off + row0, n_keys);
-        if constexpr (!SKIP) {
-          // S_x is in registers: the tensor pipe may overwrite it with the next tile
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[L::bSFree + x]);
-        }
+        // S_x is in registers: the tensor pipe may overwrite it with the next tile
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[L::bSFree + x]);
         // row maxima of the two 64-key halves (raw scores; scale > 0 commutes with max)
         float mx[2];
 #pragma unroll
@@ -847,8 +845,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // it is raised. The issuer leaves skipped halves out of P V, and the row
         // sums of the kept halves are added to l once P is handed over.
         // A warp that would drop the whole tile waits for the tile-wide decision
-        // with S still in tensor memory (S_free not yet given), so the scores
-        // need not stay in registers meanwhile; it reloads them if the tile is kept.
+        // with its scores still in registers (S_x was released at once, as in the
+        // dense kernel, so the next Q K^T is not held back by the vote).
         int vote = 0, decision = -1;
         bool skip_all = false;
         if constexpr (SKIP) {
@@ -864,11 +862,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             decision = pf_tile_decision(votes + x * 16 + (seq & 3) * 4, seq, no_abort, p.status, kWaitLimitNs);
             if (decision < 0) { ok = false; break; }
             skip_all = decision == 3;
-            if (!skip_all) pf_load_scores<CAUSAL>(taddr_s, s, key0, off + row, off + row0, n_keys);
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[L::bSFree + x]);
           if (skip_all) {
             // the whole tile is dropped: no exponentials, no P, no P V (l, O and
             // the reference stay as they are); keep the P V phase count in step
