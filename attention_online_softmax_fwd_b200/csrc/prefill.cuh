@@ -80,7 +80,8 @@ struct PrefillSmem {
   static constexpr int kBars = kRing + kStages * kTileBytes;
   // barrier indices (pairs are per query tile)
   static constexpr int bQFull = 0, bQEmpty = 2, bSFull = 4, bSFree = 6, bPFull = 8, bPVDone = 10, bOEmpty = 12,
-                       bTeardown = 14, bKVFull = 15, bKVEmpty = 15 + kStages, kNumBars = 15 + 2 * kStages;
+                       bTeardown = 14, bTurn = 15, bKVFull = 17,
+                       bKVEmpty = 17 + kStages, kNumBars = 17 + 2 * kStages;
   static constexpr int kMisc = kBars + 8 * kNumBars;            // tmem base, flags
   static constexpr int kVotes = (kMisc + 16 + 15) / 16 * 16;    // skip votes [2][4][4] ints
   static constexpr int kOrder = kMisc + 256;                    // paged: item costs and their order (below)
@@ -226,6 +227,16 @@ __device__ __forceinline__ void pf_ring_step(int step, int n, bool& is_k, int& t
   is_k = false;
   tile = m + (st - 2 * m);
 }
+
+// MUFU turns (dense and paged kernels). The two query tiles' softmax warpgroups share the
+// SM sub-partitions (warps w and w + 4 on each), and left to themselves they run in step:
+// both wait on the MUFU for their exponentials at once, then both leave it idle while
+// they load scores and store P. So on the K/V tiles that both query tiles visit they
+// take turns, passed with a pair of mbarriers of four arrivals: tile A's exponentials of
+// tile j follow tile B's of tile j - 1, and tile B's follow tile A's of tile j, so that
+// one group's exponentials overlap the other's non-MUFU work. The tile-skip kernel takes
+// no turns: there a group that drops a tile would still wait for the other's turn (and a
+// count-based hand-over that does not wait measured slower on a mostly skipped input).
 
 // Row-sum pairs (exact, as rounded for P V), added and scaled without contraction.
 __device__ __forceinline__ float2 sum2_add(float2 a, float2 b) {
@@ -395,6 +406,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&bars[L::bOEmpty + x], 4);
     }
     mbar_init(&bars[L::bTeardown], 2);
+    mbar_init(&bars[L::bTurn + 0], 4);   // tile A may take its exponentials (one arrival per tile-B warp)
+    mbar_init(&bars[L::bTurn + 1], 4);   // tile B may take its exponentials (one arrival per tile-A warp)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars[L::bKVFull + s], 1);
       mbar_init(&bars[L::bKVEmpty + s], 2);   // both MMA issuers release each slot
@@ -778,6 +791,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int own_timeout_only = 0;
     volatile int* no_abort = reinterpret_cast<volatile int*>(&own_timeout_only);
     uint32_t sf_ph = 0, pvd_ph = 0;
+    uint32_t turn_ph = 0;         // MUFU turns waited for (parity; not with the tile skip)
+    bool turn_started = false;    // this warp has taken a turn (tile A waits from its second on)
     int seq = 0;   // K/V tiles of this query tile so far (skip-vote sequence)
     bool ok = true;
 
@@ -789,6 +804,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int rows = tile_rows(qb, x);
       const int nkv = tile_nkv(qb, x, rows, off);
       if (nkv == 0) continue;
+      // K/V tiles that both query tiles of the block visit (they alternate on the MUFU there)
+      const int n_common = min(nkv, tile_nkv(qb, 1 - x, tile_rows(qb, 1 - x), off));
       const int row0 = qb * 2 * kPfRows + x * kPfRows;
       const int row = row0 + t;
       const bool row_valid = t < rows;
@@ -889,7 +906,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             alpha = (m_ref == neg_inf) ? 0.f : fast_exp2(m_ref - m_tile);
             m_ref = m_tile;
           }
-          const float offset = (m_ref == neg_inf) ? 0.f : m_ref;
+          float offset = (m_ref == neg_inf) ? 0.f : m_ref;
+          if constexpr (!SKIP) {
+            // MUFU turn: on the tiles both query tiles visit, tile A takes its exponentials
+            // after tile B's of the previous such tile, and tile B after tile A's of the same one
+            if (j < n_common && (x == 1 || turn_started)) {
+              if (!mbar_wait(&bars[L::bTurn + x], turn_ph, no_abort, p.status)) { ok = false; break; }
+              turn_ph ^= 1u;
+            }
+            asm volatile("" : "+f"(offset) : : "memory");   // no exponential before the turn
+          }
           const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
           const uint64_t negoff2 = f2_pack(-offset, -offset);
           uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -914,6 +940,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             // (P up to 2^8 under the lagging reference), the others average out.
             const float pm = fast_exp2(fmaf(mx[h], p.scale_log2, -offset));
             hsum[h].y = (mx[h] == neg_inf) ? hsum[h].x : hsum[h].x + (bf16_lo(pack_bf16x2(pm, pm)) - pm);
+          }
+          if constexpr (!SKIP) {
+            // every exponential is issued (its result is in a register) before the turn is given
+            ATTN_REG_FENCE32(pk);
+            ATTN_REG_FENCE32(pk + 32);
+            asm volatile("" : "+f"(hsum[0].y), "+f"(hsum[1].y) : : "memory");
+            if (j < n_common) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars[L::bTurn + 1 - x]);
+              turn_started = true;
+            }
           }
         }
         // P_x(j-1) must have been consumed (and O_x updated) before P_x(j) is written
