@@ -234,9 +234,15 @@ __device__ __forceinline__ void pf_ring_step(int step, int n, bool& is_k, int& t
 // they load scores and store P. So on the K/V tiles that both query tiles visit they
 // take turns, passed with a pair of mbarriers of four arrivals: tile A's exponentials of
 // tile j follow tile B's of tile j - 1, and tile B's follow tile A's of tile j, so that
-// one group's exponentials overlap the other's non-MUFU work. The tile-skip kernel takes
+// one group's exponentials overlap the other's non-MUFU work. The turn is handed on
+// after the first kTurnHandoff of the 64 exponential pairs: one warp alone keeps its
+// sub-partition's MUFU only about two-thirds busy, so the next group's first
+// exponentials fill it while this group issues its last quarter (measured best among
+// hand-overs after 32 to 64 pairs). The tile-skip kernel takes
 // no turns: there a group that drops a tile would still wait for the other's turn (and a
 // count-based hand-over that does not wait measured slower on a mostly skipped input).
+
+constexpr int kTurnHandoff = 48;
 
 // Row-sum pairs (exact, as rounded for P V), added and scaled without contraction.
 __device__ __forceinline__ float2 sum2_add(float2 a, float2 b) {
@@ -927,6 +933,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
             pk[e] = pack_bf16x2(p0, p1);
             sum2[(e / 32) * 2 + (e & 1)] = f2_add(sum2[(e / 32) * 2 + (e & 1)], f2_pack(p0, p1));
+            if constexpr (!SKIP) {
+              if (e == kTurnHandoff - 1 && j < n_common) {
+                // the first kTurnHandoff pairs are issued (their results are in registers)
+#pragma unroll
+                for (int u = 0; u < kTurnHandoff; ++u) asm volatile("" : "+r"(pk[u]) : : "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[L::bTurn + 1 - x]);
+                turn_started = true;
+              }
+            }
           }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -942,15 +958,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             hsum[h].y = (mx[h] == neg_inf) ? hsum[h].x : hsum[h].x + (bf16_lo(pack_bf16x2(pm, pm)) - pm);
           }
           if constexpr (!SKIP) {
-            // every exponential is issued (its result is in a register) before the turn is given
+            // all exponentials are in registers here (the schedule the hand-over point was chosen with)
             ATTN_REG_FENCE32(pk);
             ATTN_REG_FENCE32(pk + 32);
             asm volatile("" : "+f"(hsum[0].y), "+f"(hsum[1].y) : : "memory");
-            if (j < n_common) {
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&bars[L::bTurn + 1 - x]);
-              turn_started = true;
-            }
           }
         }
         // P_x(j-1) must have been consumed (and O_x updated) before P_x(j) is written
