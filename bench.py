@@ -666,7 +666,7 @@ def skip_overhead_report(dev, reps=5):
 
 
 PROFILE_CASES = ("skip_decode_one_pass", "skip_decode_two_pass", "dense_decode_batch", "single_seq_decode",
-                 "mha_prefill")
+                 "mha_prefill", "chunked_prefill")
 
 
 def run_profile_case(name, dev, calls=5):
@@ -678,7 +678,9 @@ def run_profile_case(name, dev, calls=5):
                             split per sequence, group decisions: two passes
       dense_decode_batch    the same 8 x 16384 tokens, dense, split 256
       single_seq_decode     the 32768-token BLASST sequence's last row, dense, split 256
-      mha_prefill           the MHA prefill B4 Hq=Hkv=32 S2048 D128, causal"""
+      mha_prefill           the MHA prefill B4 Hq=Hkv=32 S2048 D128, causal
+      chunked_prefill       the chunked prefill over 16-token pages: 4 x 2048 new tokens after
+                            cached prefixes of 0, 2048, 4096 and 6144 tokens, Hq 32 Hkv 8 D128"""
     import attention_online_softmax_fwd_b200 as ab
     scale = gen.attn_scale(128)
     ws = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
@@ -686,6 +688,10 @@ def run_profile_case(name, dev, calls=5):
         c = gen.CONFIGS["mha_prefill_llama2_7b"]
         q, k, v = [t.to(dev) for t in gen.prefill_inputs(c["B"], c["Hq"], c["Hkv"], c["S"], c["D"], c["seed"])]
         fn = lambda: ab.prefill(q, k, v, causal=True, scale=scale)
+    elif name == "chunked_prefill":
+        c = gen.paged_prefill_inputs(4, 2048, 32, 8, 128, 16, [2048, 4096, 6144, 8192], seed=1006)
+        args = [t.to(dev) for t in (c.q, c.k_pages, c.v_pages, c.block_table, c.seq_lens)]
+        fn = lambda: ab.prefill_paged(*args, scale=scale)
     else:
         if name == "skip_decode_one_pass":
             dc = gen.CONFIGS["paged_gqa_decode"]
