@@ -19,7 +19,10 @@
 // once the softmax has written the bf16 probabilities P_X(j) to shared
 // memory; the two tiles' issuers never wait on each other's softmax. So the
 // exponentials of tile j overlap the next tile's Q K^T, and the tensor pipe has
-// queued work while either softmax warpgroup computes.
+// queued work while either softmax warpgroup computes. In the dense and paged
+// kernels the two softmax warpgroups take turns on the MUFU for their
+// exponentials (the MUFU turns, below), so that one group's exponentials
+// overlap the other's score loads and P stores.
 // The exponentials use a reference maximum that is only raised when the tile
 // maximum exceeds it by more than 2^8 (exact: O and l share the reference).
 // BLASST tile skip: each softmax warp publishes a vote per 64-key half and the
