@@ -19,10 +19,10 @@
 // once the softmax has written the bf16 probabilities P_X(j) to shared
 // memory; the two tiles' issuers never wait on each other's softmax. So the
 // exponentials of tile j overlap the next tile's Q K^T, and the tensor pipe has
-// queued work while either softmax warpgroup computes. In the dense and paged
-// kernels the two softmax warpgroups take turns on the MUFU for their
-// exponentials (the MUFU turns, below), so that one group's exponentials
-// overlap the other's score loads and P stores.
+// queued work while either softmax warpgroup computes. The two softmax
+// warpgroups take turns on the MUFU for their exponentials (the MUFU turns,
+// below), so that one group's exponentials overlap the other's score loads and
+// P stores.
 // The exponentials use a reference maximum that is only raised when the tile
 // maximum exceeds it by more than 2^8 (exact: O and l share the reference).
 // BLASST tile skip: each softmax warp publishes a vote per 64-key half and the
@@ -231,7 +231,7 @@ __device__ __forceinline__ void pf_ring_step(int step, int n, bool& is_k, int& t
   tile = m + (st - 2 * m);
 }
 
-// MUFU turns (dense and paged kernels). The two query tiles' softmax warpgroups share the
+// MUFU turns. The two query tiles' softmax warpgroups share the
 // SM sub-partitions (warps w and w + 4 on each), and left to themselves they run in step:
 // both wait on the MUFU for their exponentials at once, then both leave it idle while
 // they load scores and store P. So on the K/V tiles that both query tiles visit they
@@ -241,9 +241,8 @@ __device__ __forceinline__ void pf_ring_step(int step, int n, bool& is_k, int& t
 // after the first kTurnHandoff of the 64 exponential pairs: one warp alone keeps its
 // sub-partition's MUFU only about two-thirds busy, so the next group's first
 // exponentials fill it while this group issues its last quarter (measured best among
-// hand-overs after 32 to 64 pairs). The tile-skip kernel takes
-// no turns: there a group that drops a tile would still wait for the other's turn (and a
-// count-based hand-over that does not wait measured slower on a mostly skipped input).
+// hand-overs after 32 to 64 pairs). With the tile skip, a group that drops a whole tile
+// takes the turn and hands it on at once, so that both groups count the same tiles.
 
 constexpr int kTurnHandoff = 48;
 
@@ -800,7 +799,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int own_timeout_only = 0;
     volatile int* no_abort = reinterpret_cast<volatile int*>(&own_timeout_only);
     uint32_t sf_ph = 0, pvd_ph = 0;
-    uint32_t turn_ph = 0;         // MUFU turns waited for (parity; not with the tile skip)
+    uint32_t turn_ph = 0;         // MUFU turns waited for (parity)
     bool turn_started = false;    // this warp has taken a turn (tile A waits from its second on)
     int seq = 0;   // K/V tiles of this query tile so far (skip-vote sequence)
     bool ok = true;
@@ -891,7 +890,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           if (skip_all) {
             // the whole tile is dropped: no exponentials, no P, no P V (l, O and
-            // the reference stay as they are); keep the P V phase count in step
+            // the reference stay as they are); keep the P V phase count and the
+            // MUFU turns in step (the turn is taken and handed on at once)
+            if (j < n_common) {
+              if (x == 1 || turn_started) {
+                if (!mbar_wait(&bars[L::bTurn + x], turn_ph, no_abort, p.status)) { ok = false; break; }
+                turn_ph ^= 1u;
+              }
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars[L::bTurn + 1 - x]);
+              turn_started = true;
+            }
             if (j > 0) {
               if (!mbar_wait(&bars[L::bPVDone + x], pvd_ph, no_abort, p.status)) { ok = false; break; }
               pvd_ph ^= 1u;
@@ -916,7 +925,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             m_ref = m_tile;
           }
           float offset = (m_ref == neg_inf) ? 0.f : m_ref;
-          if constexpr (!SKIP) {
+          {
             // MUFU turn: on the tiles both query tiles visit, tile A takes its exponentials
             // after tile B's of the previous such tile, and tile B after tile A's of the same one
             if (j < n_common && (x == 1 || turn_started)) {
@@ -936,7 +945,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
             pk[e] = pack_bf16x2(p0, p1);
             sum2[(e / 32) * 2 + (e & 1)] = f2_add(sum2[(e / 32) * 2 + (e & 1)], f2_pack(p0, p1));
-            if constexpr (!SKIP) {
+            {
               if (e == kTurnHandoff - 1 && j < n_common) {
                 // the first kTurnHandoff pairs are issued (their results are in registers)
 #pragma unroll

@@ -1,4 +1,4 @@
-"""Host model of the prefill kernel's MUFU turns (prefill.cuh, dense and paged kernels).
+"""Host model of the prefill kernel's MUFU turns (prefill.cuh; dense, paged and tile-skip kernels).
 
 The two softmax warpgroups of a CTA (query tiles A and B of each 256-row block) take
 turns for their exponentials on the K/V tiles both visit: tile A's exponentials of
